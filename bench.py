@@ -1,0 +1,481 @@
+"""Benchmark: one streaming LCSA step per 8-frame chunk at 768x1408 on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload chunk|multistream|uhr_truncate|uhr_preserve|clip|clip_5|clip_30]
+
+A step is the whole hot path over one chunk: lcsa_pool_qk (Q and the new K),
+lcsa_kv_append (K, V, pooled K into the ring cache, evicting the oldest
+frames), lcsa_select_blocks (coarse map, causal mask, top-K) and
+lcsa_sparse_attn_fwd, with Q/K/V resident in HBM. L2 is flushed (a 512 MB
+write) before every timed step, outside the timed events. Under torchrun each
+rank streams its own independent video (weak scaling, no data-path
+collective); the step time is the max over ranks.
+
+Rank 0 prints one JSON line. `--impl reference` times the fp64 CPU oracle on
+a bounded sample of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import lcsa_inputs as li  # noqa: E402
+
+METRIC = "ms per 8-frame chunk at 768x1408; sparse-attn TFLOP/s and % of BF16/HBM roofline"
+UNIT = "ms/chunk"
+CHUNKS_PER_STEP = {"clip": 13, "clip_5": 13, "clip_30": 13}  # a whole clip is 13 two-frame chunks
+
+WORKLOAD_TEXT = {
+    "chunk": "768x1408 streaming chunk: 12 heads, d=128, 48x88 tokens/frame, 2-frame query chunk "
+             "vs 6-frame KV cache (chunk + 4 past), 3D RoPE, 13.6% of causal block pairs",
+    "multistream": "4 streams at 768x1408, 2-frame chunks, ragged 4/5/6 past frames, 13.6%",
+    "uhr_truncate": "1536x2688: 96x168 tokens/frame, 2+4 frames, 9x9-block window, truncate, 13.6%",
+    "uhr_preserve": "1536x2688: 96x168 tokens/frame, 2+4 frames, 9x9-block window, preserve, 13.6%",
+    "clip": "whole 101-frame clip at 768x1408: 26 latent frames, block-causal, 13.6%",
+    "clip_5": "whole 101-frame clip at 768x1408: 26 latent frames, block-causal, 5%",
+    "clip_30": "whole 101-frame clip at 768x1408: 26 latent frames, block-causal, 30%",
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [s.strip() for s in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def attn_flops(blk_cnt: torch.Tensor, blk_idx: torch.Tensor, cache, Hb: int, Wb: int, D: int,
+               q_tokens_per_block: int = 128) -> float:
+    """4*D*sum(q tokens x kept key tokens); a one-frame key block counts 64 keys."""
+    cnt = blk_cnt.long().cpu()
+    idx = blk_idx.long().cpu()
+    total = 0
+    for b in range(cnt.shape[0]):
+        keys = cnt[b].sum().item() * 128
+        if cache.begin(b) % 2 == 1:  # oldest cached block has one frame
+            valid = torch.arange(idx.shape[-1]).view(1, 1, -1) < cnt[b].unsqueeze(-1)
+            n_partial = ((idx[b] < Hb * Wb) & (idx[b] >= 0) & valid).sum().item()
+            keys -= 64 * n_partial
+        total += keys
+    return 4.0 * D * q_tokens_per_block * total
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, world, rank, local):
+    import block_sparse_causal_lcsa_b200 as lc
+
+    w = li.workload(args.workload)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    # each rank streams an independent video (weak scaling)
+    w = li.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+    streaming = w.kv_past[0] > 0 or w.B > 1
+    x = li.make_inputs(w)
+    params = lc.SelectParams(top_k=w.top_k, density=w.density, window=w.window,
+                             window_mode=w.window_mode)
+    n_chunks = 3
+    if streaming:
+        cache = lc.KVCache(w.B, w.H, w.cap_frames, w.Y, w.X, w.D, device=dev)
+        for b in range(w.B):
+            kp = x["k"][b][:, :w.kv_past[b]].unsqueeze(0).to(dev)
+            vp = x["v"][b][:, :w.kv_past[b]].unsqueeze(0).to(dev)
+            lc.kv_append(cache, kp, vp, lc.pool_qk(kp)[0], stream_offset=b)
+        # distinct chunks cycled through the steps (the stream keeps advancing)
+        g = torch.Generator().manual_seed(w.seed + 7)
+        shp = (w.B, w.H, w.q_frames, w.Y, w.X, w.D)
+        chunks = [(x["q"].to(dev),
+                   torch.stack([x["k"][b][:, -w.q_frames:] for b in range(w.B)]).to(dev),
+                   torch.stack([x["v"][b][:, -w.q_frames:] for b in range(w.B)]).to(dev))]
+        for _ in range(n_chunks - 1):
+            chunks.append(tuple(torch.randn(shp, generator=g).to(torch.bfloat16).to(dev)
+                                for _ in range(3)))
+        step = lc.StreamingStep(cache, w.q_frames, params)
+        base_state = cache.state()
+
+        def run_step(i, q=None, k=None, v=None, ev=None):
+            if q is None:
+                q, k, v = chunks[i % n_chunks]
+            # every step sees the workload's cache lengths (host-side state only);
+            # the append still writes 2 frames and the pooled K into the ring
+            step.cache.set_state(base_state)
+            if ev is not None:
+                ev[0].record()
+            lc.pool_qk(q, k, step.q_pool, step.k_pool)
+            if ev is not None:
+                ev[1].record()
+            lc.kv_append(step.cache, k, v, step.k_pool)
+            if ev is not None:
+                ev[2].record()
+            lc.select_blocks(step.q_pool, step.q_frames, step.cache, step.params, step.kmax,
+                             step.blk_idx, step.blk_cnt)
+            if ev is not None:
+                ev[3].record()
+            lc.sparse_attn_fwd(q, step.cache, step.blk_idx, step.blk_cnt, step.o, step.lse)
+            if ev is not None:
+                ev[4].record()
+            return step.o
+
+        kernels = ["pool", "kv_append", "select", "attn"]
+        q_frames_step = w.q_frames
+        sel_ref = step
+    else:
+        # whole clip: Q, K, V of all frames resident; no append
+        q = x["q"].to(dev)
+        k = x["k"][0].unsqueeze(0).to(dev)
+        v = x["v"][0].unsqueeze(0).to(dev)
+        q_pool = torch.empty(lc.api.pooled_shape(q), dtype=torch.float64, device=dev)
+        k_pool = torch.empty(lc.api.pooled_shape(k), dtype=torch.float64, device=dev)
+        cache = lc.KVCache.wrap(k, v, k_pool)
+        kmax = lc.select_kmax(cache, w.q_frames, params)
+        nQB = q_pool.shape[2] * q_pool.shape[3] * q_pool.shape[4]
+        blk_idx = torch.empty((1, w.H, nQB, kmax), dtype=torch.int32, device=dev)
+        blk_cnt = torch.empty((1, w.H, nQB), dtype=torch.int32, device=dev)
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:5], dtype=torch.float32, device=dev)
+        base_state = cache.state()
+
+        class _S:
+            pass
+        sel_ref = _S()
+        sel_ref.blk_idx, sel_ref.blk_cnt, sel_ref.o = blk_idx, blk_cnt, o
+
+        def run_step(i, qq=None, kk=None, vv=None, ev=None):
+            if ev is not None:
+                ev[0].record()
+            lc.pool_qk(q, k, q_pool, k_pool)
+            if ev is not None:
+                ev[1].record()
+            lc.select_blocks(q_pool, w.q_frames, cache, params, kmax, blk_idx, blk_cnt)
+            if ev is not None:
+                ev[2].record()
+            lc.sparse_attn_fwd(q, cache, blk_idx, blk_cnt, o, lse)
+            if ev is not None:
+                ev[3].record()
+            return o
+
+        kernels = ["pool", "select", "attn"]
+        q_frames_step = w.q_frames
+
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for i in range(args.warmup):
+        flush.zero_()
+        run_step(i)
+    torch.cuda.synchronize()
+    if lc.last_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    nev = len(kernels) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        run_step(args.warmup + i, ev=evs[i])
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    barrier(world)
+    time.sleep(0.2)
+    clk = clocks.stop()
+    if lc.last_device_error() != 0:
+        raise RuntimeError("device error during the timed steps")
+    step_ms = [evs[i][0].elapsed_time(evs[i][-1]) for i in range(args.steps)]
+    per_kernel = {kname: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+                  for j, kname in enumerate(kernels)}
+    mean_step = statistics.mean(step_ms)
+    mean_step_max = max_over_ranks(mean_step, world)
+    chunks_per_step = CHUNKS_PER_STEP.get(args.workload, 1) * w.B
+    value = mean_step_max / (chunks_per_step * world)
+
+    flops = attn_flops(sel_ref.blk_cnt, sel_ref.blk_idx, cache, w.Hb, w.Wb, w.D)
+    attn_s = per_kernel["attn"] / 1e3
+    achieved_tflops = flops / attn_s / 1e12
+    peak = peaks["bf16_tflops"]
+
+    # e2e: the same step through the API with inputs from pinned host memory and
+    # the output read back, copies inside the timed region
+    e2e = None
+    if streaming:
+        hq = chunks[0][0].cpu().pin_memory()
+        hk = chunks[0][1].cpu().pin_memory()
+        hv = chunks[0][2].cpu().pin_memory()
+        ho = torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory()
+        dq, dk, dv = torch.empty_like(chunks[0][0]), torch.empty_like(chunks[0][1]), torch.empty_like(chunks[0][2])
+        e_start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        e_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            if i >= args.warmup:
+                e_start[i - args.warmup].record()
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            out = run_step(i, dq, dk, dv)
+            ho.copy_(out, non_blocking=True)
+            if i >= args.warmup:
+                e_end[i - args.warmup].record()
+        torch.cuda.synchronize()
+        e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(e_start, e_end))
+        e2e_ms = max_over_ranks(e2e_ms, world)
+        e2e = {"value": e2e_ms / (chunks_per_step * world), "unit": UNIT,
+               "h2d_bytes_per_step": hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2,
+               "d2h_bytes_per_step": ho.numel() * 2}
+    else:
+        hq = q.cpu().pin_memory()
+        hk = k.cpu().pin_memory()
+        hv = v.cpu().pin_memory()
+        ho = torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory()
+        e_start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        e_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.warmup + args.steps):
+            if i >= args.warmup:
+                e_start[i - args.warmup].record()
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            out = run_step(i)
+            ho.copy_(out, non_blocking=True)
+            if i >= args.warmup:
+                e_end[i - args.warmup].record()
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(e_start, e_end)), world)
+        e2e = {"value": e2e_ms / (chunks_per_step * world), "unit": UNIT,
+               "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel()) * 2,
+               "d2h_bytes_per_step": ho.numel() * 2}
+    if lc.last_device_error() != 0:
+        raise RuntimeError("device error during the end-to-end steps")
+
+    # HBM-side kernels: algorithmic bytes per launch
+    tokens_q = w.B * w.H * q_frames_step * w.Y * w.X
+    # pool reads Q and the new K (bf16) once and writes one float64 row per block
+    bytes_pool = 2 * tokens_q * w.D * 2 + 2 * (tokens_q // 128) * w.D * 8
+    hbm = {"pool_gbs": bytes_pool / (per_kernel["pool"] / 1e3) / 1e9}
+    if "kv_append" in per_kernel:
+        bytes_app = 2 * (2 * tokens_q * w.D * 2) + 2 * (tokens_q // 128) * w.D * 8
+        hbm["kv_append_gbs"] = bytes_app / (per_kernel["kv_append"] / 1e3) / 1e9
+
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "attn_traffic_%s.json" % args.workload)
+    if os.path.exists(tfile):
+        traffic = json.load(open(tfile)).get("bytes_per_launch")
+
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(mean_step_max, 4),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, shapes of the pages' 768x1408 workload)",
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload,
+                   "streams_per_gpu": w.B, "heads": w.H, "head_dim": w.D,
+                   "tokens_per_frame": w.Y * w.X, "q_frames": w.q_frames,
+                   "kv_frames": list(w.kv_frames), "density": w.density, "window": w.window,
+                   "l2": "flushed before every timed step (512 MB write)",
+                   "select_precision": "fp64 scores, exact top-K",
+                   "parallelism": "independent stream per GPU" if world > 1 else "single GPU"},
+        "per_kernel_ms": {k2: round(v2, 5) for k2, v2 in per_kernel.items()},
+        "sparse_attn_tflops": round(achieved_tflops, 2),
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd", "achieved": round(achieved_tflops, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved_tflops / peak, 4),
+                     "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % peaks["source"],
+                     "flops_per_launch": flops, "traffic": traffic},
+        "hbm_kernels": {k2: round(v2, 1) for k2, v2 in hbm.items()},
+        "hbm_peak_gbs": peaks["hbm_gbs"],
+        "e2e": e2e,
+        "gpu_launches": len(kernels) * args.steps,
+        "clocks": clk,
+        "wall_s_timed": round(t_wall, 4),
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, x, budget_s=args.cpu_budget)
+    return line
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 1) for p in threadpool_info()]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, x, budget_s=15.0):
+    """The fp64 oracle as it stands, on whole heads of the workload until the
+    budget is spent; scaled to ms per chunk."""
+    from oracle import lcsa_oracle as orc
+
+    t0 = time.perf_counter()
+    done = 0
+    streams = [(b, h) for b in range(w.B) for h in range(w.H)]
+    for b, h in streams:
+        orc.lcsa_head(orc.widen(x["q"][b, h]), orc.widen(x["k"][b][h]), orc.widen(x["v"][b][h]),
+                      top_k=w.top_k, density=w.density, window=w.window, mode=w.window_mode)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    el = time.perf_counter() - t0
+    per_chunk_ms = el / done * len(streams) / (CHUNKS_PER_STEP.get(w.name, 1) * w.B) * 1e3
+    return {"value": round(per_chunk_ms, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": "%d of %d (stream, head) units of the workload, whole path (pool, select, "
+                      "attention) in fp64, scaled to the full chunk" % (done, len(streams))}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    w = li.workload(args.workload)
+    x = li.make_inputs(w)
+    from oracle import lcsa_oracle as orc
+
+    units = [(b, h) for b in range(w.B) for h in range(w.H)]
+    times = []
+    for i in range(args.warmup + args.steps):
+        b, h = units[i % len(units)]
+        t0 = time.perf_counter()
+        orc.lcsa_head(orc.widen(x["q"][b, h]), orc.widen(x["k"][b][h]), orc.widen(x["v"][b][h]),
+                      top_k=w.top_k, density=w.density, window=w.window, mode=w.window_mode)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    per_chunk_ms = statistics.mean(times) * len(units) / (CHUNKS_PER_STEP.get(args.workload, 1) * w.B) * 1e3
+    sample = ("one (stream, head) unit per step, whole path (pool, select, attention) in fp64, "
+              "scaled by %d units to the full chunk" % len(units))
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(per_chunk_ms, 2), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(statistics.mean(times) * 1e3, 2), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload},
+        "cpu_baseline": {"value": round(per_chunk_ms, 2), "unit": UNIT, "cores": _threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(per_chunk_ms, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="chunk", choices=sorted(WORKLOAD_TEXT))
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        line = run_ours(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,25 @@
+"""B200 (sm_100a) locality-constrained block-sparse causal attention.
+
+FlashVSR's LCSA attention core as a C-ABI CUDA library (liblcsa.so, declared
+in include/lcsa.h) with a thin PyTorch binding: block pooling, block
+selection (causal + locality window + top-K), tcgen05 sparse attention and
+the streaming KV-cache append.
+"""
+from .api import (  # noqa: F401
+    KVCache,
+    LcsaError,
+    SelectParams,
+    StreamingStep,
+    WINDOW_PRESERVE,
+    WINDOW_TRUNCATE,
+    debug_set_wait_limit_ns,
+    debug_stalled_wait,
+    kv_append,
+    last_device_error,
+    pool_qk,
+    select_blocks,
+    select_kmax,
+    sparse_attn_fwd,
+    tensor_desc,
+)
+from .build import LIB_PATH  # noqa: F401

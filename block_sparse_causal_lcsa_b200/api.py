@@ -1,0 +1,254 @@
+"""PyTorch-facing binding of liblcsa.so.
+
+Each function takes torch CUDA tensors, marshals their pointers, extents and
+strides into the C structs of include/lcsa.h and calls the entry point of the
+same name on the current torch stream. Output buffers are allocated with torch
+when the caller does not pass them (the library itself allocates nothing).
+No step of the attention path runs here: there is no CPU fallback, and a
+missing or incomplete liblcsa.so raises ImportError at import.
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+import torch
+
+from . import _abi
+
+_lib = _abi.load()
+
+OK = _abi.OK
+WINDOW_TRUNCATE = _abi.WINDOW_TRUNCATE
+WINDOW_PRESERVE = _abi.WINDOW_PRESERVE
+TIE_EPS = 1e-5
+
+
+class LcsaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        msg = _lib.lcsa_status_string(status).decode()
+        super().__init__("%s: %s (status %d)" % (what, msg, status) if what else msg)
+
+
+def _check(status: int, what: str) -> None:
+    if status != OK:
+        raise LcsaError(status, what)
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def tensor_desc(x: torch.Tensor) -> _abi.Tensor:
+    """lcsa_tensor for a bf16 tensor of shape [B][H][T][Y][X][D] (D unit stride)."""
+    if x.dim() != 6 or x.dtype != torch.bfloat16 or not x.is_cuda:
+        raise ValueError("expected a CUDA bf16 tensor [B][H][T][Y][X][D]")
+    if x.stride(5) != 1:
+        raise ValueError("the channel dimension must have unit stride")
+    B, H, T, Y, X, D = x.shape
+    sb, sh, st, sy, sx, _ = x.stride()
+    return _abi.Tensor(x.data_ptr(), B, H, T, Y, X, D, sb, sh, st, sy, sx)
+
+
+def pooled_shape(x: torch.Tensor) -> Tuple[int, ...]:
+    B, H, T, Y, X, D = x.shape
+    return (B, H, (T + 1) // 2, Y // 8, X // 8, D)
+
+
+def pool_qk(q: torch.Tensor, k: Optional[torch.Tensor] = None,
+            q_pool: Optional[torch.Tensor] = None, k_pool: Optional[torch.Tensor] = None,
+            stream: Optional[torch.cuda.Stream] = None):
+    """Mean-pool Q (and K) over 2x8x8 token blocks into float64 features."""
+    if q_pool is None:
+        q_pool = torch.empty(pooled_shape(q), dtype=torch.float64, device=q.device)
+    if k is not None and k_pool is None:
+        k_pool = torch.empty(pooled_shape(k), dtype=torch.float64, device=k.device)
+    qd = tensor_desc(q)
+    kd = tensor_desc(k) if k is not None else None
+    _check(_lib.lcsa_pool_qk(C.byref(qd), C.byref(kd) if kd is not None else None,
+                             q_pool.data_ptr(), k_pool.data_ptr() if k is not None else None,
+                             _stream(stream)), "lcsa_pool_qk")
+    return q_pool, k_pool
+
+
+class KVCache:
+    """Streaming ring cache of K, V and pooled K for B streams (device buffers
+    owned by this object, begin/end state kept host-side in the C struct)."""
+
+    def __init__(self, B: int, H: int, cap_frames: int, Y: int, X: int, D: int,
+                 device="cuda", k: torch.Tensor = None, v: torch.Tensor = None,
+                 k_pool: torch.Tensor = None):
+        shape = (B, H, cap_frames, Y, X, D)
+        self.k = k if k is not None else torch.empty(shape, dtype=torch.bfloat16, device=device)
+        self.v = v if v is not None else torch.empty(shape, dtype=torch.bfloat16, device=device)
+        self.k_pool = (k_pool if k_pool is not None else
+                       torch.empty((B, H, cap_frames // 2, Y // 8, X // 8, D), dtype=torch.float64,
+                                   device=device))
+        for t in (self.k, self.v, self.k_pool):
+            if not t.is_contiguous():
+                raise ValueError("cache buffers must be contiguous")
+        self.struct = _abi.KVCacheStruct()
+        self.struct.k = self.k.data_ptr()
+        self.struct.v = self.v.data_ptr()
+        self.struct.k_pool = self.k_pool.data_ptr()
+        self.struct.B, self.struct.H, self.struct.cap_frames = B, H, cap_frames
+        self.struct.Y, self.struct.X, self.struct.D = Y, X, D
+        self.B, self.H, self.cap_frames, self.Y, self.X, self.D = B, H, cap_frames, Y, X, D
+
+    @classmethod
+    def wrap(cls, k: torch.Tensor, v: torch.Tensor, k_pool: torch.Tensor) -> "KVCache":
+        """View whole K/V sequences [B][H][F][Y][X][D] (F even) as a full cache."""
+        B, H, F, Y, X, D = k.shape
+        c = cls(B, H, F, Y, X, D, k=k.contiguous(), v=v.contiguous(), k_pool=k_pool.contiguous())
+        for b in range(B):
+            c.struct.begin[b] = 0
+            c.struct.end[b] = F
+        return c
+
+    def begin(self, b: int) -> int:
+        return int(self.struct.begin[b])
+
+    def end(self, b: int) -> int:
+        return int(self.struct.end[b])
+
+    def frames(self, b: int) -> int:
+        return self.end(b) - self.begin(b)
+
+    def reset(self) -> None:
+        for b in range(self.B):
+            self.struct.begin[b] = 0
+            self.struct.end[b] = 0
+
+    def state(self):
+        return [(self.begin(b), self.end(b)) for b in range(self.B)]
+
+    def set_state(self, state) -> None:
+        for b, (lo, hi) in enumerate(state):
+            self.struct.begin[b] = lo
+            self.struct.end[b] = hi
+
+
+def kv_append(cache: KVCache, k_new: torch.Tensor, v_new: torch.Tensor, k_pool_new: torch.Tensor,
+              stream_offset: int = 0, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Append a chunk (and its pooled K) to streams [offset, offset+B) of the cache."""
+    kd, vd = tensor_desc(k_new), tensor_desc(v_new)
+    if not k_pool_new.is_contiguous() or k_pool_new.dtype != torch.float64:
+        raise ValueError("k_pool_new must be contiguous float64")
+    _check(_lib.lcsa_kv_append(C.byref(cache.struct), C.byref(kd), C.byref(vd),
+                               k_pool_new.data_ptr(), stream_offset, _stream(stream)),
+           "lcsa_kv_append")
+
+
+@dataclass
+class SelectParams:
+    top_k: int = 0
+    density: float = 0.0
+    window: int = 0
+    window_mode: int = WINDOW_TRUNCATE
+    tie_eps: float = TIE_EPS
+
+    def struct(self, kmax: int = 0) -> _abi.SelectParamsStruct:
+        return _abi.SelectParamsStruct(self.top_k, self.window, self.window_mode, kmax,
+                                       float(self.density), float(self.tie_eps))
+
+
+def select_kmax(cache: KVCache, q_frames: int, params: SelectParams) -> int:
+    sp = params.struct()
+    return int(_lib.lcsa_select_kmax(C.byref(cache.struct), q_frames, C.byref(sp)))
+
+
+def select_blocks(q_pool: torch.Tensor, q_frames: int, cache: KVCache, params: SelectParams,
+                  kmax: Optional[int] = None, blk_idx: Optional[torch.Tensor] = None,
+                  blk_cnt: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None):
+    """Top-K key blocks of every query block: (blk_idx [B,H,nQB,kmax], blk_cnt [B,H,nQB])."""
+    if kmax is None:
+        kmax = select_kmax(cache, q_frames, params)
+    B, H, nQT, Hb, Wb, D = q_pool.shape
+    if not q_pool.is_contiguous() or q_pool.dtype != torch.float64:
+        raise ValueError("q_pool must be contiguous float64")
+    nQB = nQT * Hb * Wb
+    if blk_idx is None:
+        blk_idx = torch.empty((B, H, nQB, kmax), dtype=torch.int32, device=q_pool.device)
+    if blk_cnt is None:
+        blk_cnt = torch.empty((B, H, nQB), dtype=torch.int32, device=q_pool.device)
+    sp = params.struct(kmax)
+    _check(_lib.lcsa_select_blocks(q_pool.data_ptr(), q_frames, C.byref(cache.struct), C.byref(sp),
+                                   blk_idx.data_ptr(), blk_cnt.data_ptr(), _stream(stream)),
+           "lcsa_select_blocks")
+    return blk_idx, blk_cnt
+
+
+def sparse_attn_fwd(q: torch.Tensor, cache: KVCache, blk_idx: torch.Tensor, blk_cnt: torch.Tensor,
+                    o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                    with_lse: bool = True, stream: Optional[torch.cuda.Stream] = None):
+    """Attention of the query chunk over its kept key blocks: (O bf16 like q, LSE fp32)."""
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and with_lse:
+        lse = torch.empty(q.shape[:5], dtype=torch.float32, device=q.device)
+    if not blk_idx.is_contiguous() or not blk_cnt.is_contiguous():
+        raise ValueError("blk_idx and blk_cnt must be contiguous")
+    qd, od = tensor_desc(q), tensor_desc(o)
+    _check(_lib.lcsa_sparse_attn_fwd(C.byref(qd), C.byref(cache.struct), blk_idx.data_ptr(),
+                                     blk_cnt.data_ptr(), blk_idx.shape[-1], C.byref(od),
+                                     lse.data_ptr() if lse is not None else None, _stream(stream)),
+           "lcsa_sparse_attn_fwd")
+    return o, lse
+
+
+def last_device_error(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronise the stream, read and clear the device error word (status code)."""
+    return int(_lib.lcsa_last_device_error(_stream(stream)))
+
+
+def debug_stalled_wait(limit_ns: int, stream: Optional[torch.cuda.Stream] = None) -> None:
+    _check(_lib.lcsa_debug_stalled_wait(limit_ns, _stream(stream)), "lcsa_debug_stalled_wait")
+
+
+def debug_set_wait_limit_ns(ns: int) -> None:
+    _check(_lib.lcsa_debug_set_wait_limit_ns(ns), "lcsa_debug_set_wait_limit_ns")
+
+
+class StreamingStep:
+    """One streaming LCSA step over preallocated buffers: pool Q and the new K,
+    append K/V and pooled K to the cache, select the top-K blocks, attend.
+
+    The four library calls are the whole step; buffers are allocated once here
+    so that repeated steps launch kernels only.
+    """
+
+    def __init__(self, cache: KVCache, q_frames: int, params: SelectParams, new_frames: int = None):
+        self.cache = cache
+        self.q_frames = q_frames
+        self.params = params
+        dev = cache.k.device
+        B, H, Y, X, D = cache.B, cache.H, cache.Y, cache.X, cache.D
+        nf = q_frames if new_frames is None else new_frames
+        nQT = (q_frames + 1) // 2
+        self.q_pool = torch.empty((B, H, nQT, Y // 8, X // 8, D), dtype=torch.float64, device=dev)
+        self.k_pool = torch.empty((B, H, (nf + 1) // 2, Y // 8, X // 8, D), dtype=torch.float64,
+                                  device=dev)
+        # capacity for the fullest cache state this step can see
+        full = _abi.KVCacheStruct.from_buffer_copy(cache.struct)
+        for b in range(B):
+            full.begin[b], full.end[b] = 0, cache.cap_frames
+        sp = params.struct()
+        self.kmax = int(_lib.lcsa_select_kmax(C.byref(full), q_frames, C.byref(sp)))
+        nQB = nQT * (Y // 8) * (X // 8)
+        self.blk_idx = torch.empty((B, H, nQB, self.kmax), dtype=torch.int32, device=dev)
+        self.blk_cnt = torch.empty((B, H, nQB), dtype=torch.int32, device=dev)
+        self.o = torch.empty((B, H, q_frames, Y, X, D), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((B, H, q_frames, Y, X), dtype=torch.float32, device=dev)
+
+    def __call__(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                 stream: Optional[torch.cuda.Stream] = None):
+        pool_qk(q, k_new, self.q_pool, self.k_pool, stream)
+        kv_append(self.cache, k_new, v_new, self.k_pool, 0, stream)
+        select_blocks(self.q_pool, self.q_frames, self.cache, self.params, self.kmax,
+                      self.blk_idx, self.blk_cnt, stream)
+        sparse_attn_fwd(q, self.cache, self.blk_idx, self.blk_cnt, self.o, self.lse, stream=stream)
+        return self.o, self.lse

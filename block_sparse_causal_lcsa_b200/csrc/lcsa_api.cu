@@ -1,0 +1,434 @@
+// Host side of liblcsa.so: the C ABI declared in include/lcsa.h. Validates
+// every argument before launching, encodes the TMA tensor maps, sizes the
+// grids and launches the sm_100a kernels on the caller's stream. Allocates no
+// memory: the only device state of the library is its per-device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "lcsa.h"
+#include "attn_fwd.cuh"
+#include "kv_append.cuh"
+#include "pool.cuh"
+#include "select.cuh"
+
+namespace lcsa {
+
+// Error word shared by all kernels of this library on one device.
+__device__ unsigned int g_device_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultWaitNs = 1000000000ull;  // 1 s
+uint64_t g_wait_limit_ns = kDefaultWaitNs;
+
+std::mutex g_mu;
+unsigned int* g_err_ptr[kMaxDevices] = {};
+bool g_attr_done[kMaxDevices] = {};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Current device, its error-word address and one-time kernel attributes.
+lcsa_status device_setup(int* dev_out, unsigned int** err_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LCSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_err_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_device_error) != cudaSuccess) return LCSA_ERR_CUDA;
+    g_err_ptr[dev] = static_cast<unsigned int*>(ptr);
+  }
+  if (!g_attr_done[dev]) {
+    if (cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnLayout<128>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnLayout<64>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             227 * 1024) != cudaSuccess)
+      return LCSA_ERR_CUDA;
+    g_attr_done[dev] = true;
+  }
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return LCSA_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  *dev_out = dev;
+  *err_out = g_err_ptr[dev];
+  return LCSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks common to every token tensor.
+lcsa_status check_tensor(const lcsa_tensor* t) {
+  if (t == nullptr || t->data == nullptr) return LCSA_ERR_INVALID_ARG;
+  if (t->B < 1 || t->H < 1 || t->T < 1 || t->Y < 8 || t->X < 8) return LCSA_ERR_SHAPE;
+  if (t->D != 64 && t->D != 128) return LCSA_ERR_SHAPE;
+  if (t->Y % 8 || t->X % 8) return LCSA_ERR_SHAPE;
+  if (t->B > LCSA_MAX_STREAMS) return LCSA_ERR_SHAPE;
+  if (!aligned16(t->data)) return LCSA_ERR_ALIGN;
+  const int64_t s[5] = {t->stride_b, t->stride_h, t->stride_t, t->stride_y, t->stride_x};
+  for (int i = 0; i < 5; ++i)
+    if (s[i] <= 0 || s[i] % 8) return LCSA_ERR_ALIGN;
+  if (t->stride_b != static_cast<int64_t>(t->H) * t->stride_h) return LCSA_ERR_SHAPE;
+  if (t->stride_x < t->D) return LCSA_ERR_SHAPE;
+  return LCSA_OK;
+}
+
+lcsa_status check_cache(const lcsa_kv_cache* kv) {
+  if (kv == nullptr || kv->k == nullptr || kv->v == nullptr || kv->k_pool == nullptr)
+    return LCSA_ERR_INVALID_ARG;
+  if (kv->B < 1 || kv->B > LCSA_MAX_STREAMS || kv->H < 1) return LCSA_ERR_SHAPE;
+  if (kv->D != 64 && kv->D != 128) return LCSA_ERR_SHAPE;
+  if (kv->Y < 8 || kv->X < 8 || kv->Y % 8 || kv->X % 8) return LCSA_ERR_SHAPE;
+  if (kv->cap_frames < 2 || kv->cap_frames % 2) return LCSA_ERR_SHAPE;
+  if (!aligned16(kv->k) || !aligned16(kv->v) || !aligned16(kv->k_pool)) return LCSA_ERR_ALIGN;
+  for (int b = 0; b < kv->B; ++b) {
+    const int64_t n = kv->end[b] - kv->begin[b];
+    if (kv->begin[b] < 0 || n < 0 || n > kv->cap_frames || (kv->end[b] & 1)) return LCSA_ERR_INVALID_ARG;
+  }
+  return LCSA_OK;
+}
+
+int temporal_blocks(int frames) { return (frames + 1) / 2; }
+
+// 5-D map (d, x, y, frame, stream*head) over bf16 tokens; box = 64 channels x
+// 8 x 8 tokens x 1 frame, 128-byte swizzle.
+lcsa_status encode_map(CUtensorMap* map, void* data, int B, int H, int T, int Y, int X, int D,
+                       int64_t sh, int64_t st, int64_t sy, int64_t sx) {
+  const cuuint64_t dims[5] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(X),
+                              static_cast<cuuint64_t>(Y), static_cast<cuuint64_t>(T),
+                              static_cast<cuuint64_t>(B) * H};
+  const cuuint64_t strides[4] = {static_cast<cuuint64_t>(sx) * 2, static_cast<cuuint64_t>(sy) * 2,
+                                 static_cast<cuuint64_t>(st) * 2, static_cast<cuuint64_t>(sh) * 2};
+  const cuuint32_t box[5] = {64, 8, 8, 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, data, dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LCSA_OK : LCSA_ERR_CUDA;
+}
+
+// One thread waits on a barrier that nothing arrives at: the bounded wait
+// must give up, set the error word and return (test of the timeout path).
+__global__ void stalled_wait_kernel(uint64_t limit_ns, unsigned int* err) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    mbar_init_fence();
+    const WaitCtx w{limit_ns, &abort_flag, err};
+    wait_bounded(smem_u32(&bar), 0, w);
+  }
+}
+
+lcsa_status launched() { return cudaGetLastError() == cudaSuccess ? LCSA_OK : LCSA_ERR_CUDA; }
+
+// K_i upper bound over the rows of a selection (largest C_i gives largest K_i).
+int32_t kmax_for(int nKT, int nQT, int Hb, int Wb, const lcsa_select_params* p) {
+  if (nKT < nQT || nQT < 1) return 0;
+  int wy = Hb, wx = Wb;
+  if (p->window > 0) {
+    wy = p->window < Hb ? p->window : Hb;
+    wx = p->window < Wb ? p->window : Wb;
+  }
+  const int C = nKT * wy * wx;
+  if (p->top_k > 0) return p->top_k < C ? p->top_k : C;
+  int K = static_cast<int>(std::ceil(p->density * static_cast<double>(C)));
+  if (K < 1) K = 1;
+  return K < C ? K : C;
+}
+
+}  // namespace
+}  // namespace lcsa
+
+using namespace lcsa;
+
+extern "C" {
+
+int32_t lcsa_abi_version(void) { return LCSA_ABI_VERSION; }
+
+const char* lcsa_status_string(lcsa_status s) {
+  switch (s) {
+    case LCSA_OK: return "ok";
+    case LCSA_ERR_INVALID_ARG: return "invalid argument";
+    case LCSA_ERR_SHAPE: return "unsupported or inconsistent shape";
+    case LCSA_ERR_ALIGN: return "misaligned pointer or stride";
+    case LCSA_ERR_CAPACITY: return "capacity exceeded";
+    case LCSA_ERR_WORKSPACE: return "workspace error";
+    case LCSA_ERR_CUDA: return "CUDA error";
+    case LCSA_ERR_TIMEOUT: return "a kernel wait timed out";
+    case LCSA_ERR_DEVICE_BOUNDS: return "a kernel saw an out-of-range block id";
+  }
+  return "unknown status";
+}
+
+lcsa_status lcsa_pool_qk(const lcsa_tensor* q, const lcsa_tensor* k, double* q_pool, double* k_pool,
+                         lcsa_stream_t stream) {
+  lcsa_status s = check_tensor(q);
+  if (s != LCSA_OK) return s;
+  if (q_pool == nullptr || !aligned16(q_pool)) return q_pool ? LCSA_ERR_ALIGN : LCSA_ERR_INVALID_ARG;
+  if (k != nullptr) {
+    if ((s = check_tensor(k)) != LCSA_OK) return s;
+    if (k->B != q->B || k->H != q->H || k->Y != q->Y || k->X != q->X || k->D != q->D) return LCSA_ERR_SHAPE;
+    if (k_pool == nullptr || !aligned16(k_pool)) return k_pool ? LCSA_ERR_ALIGN : LCSA_ERR_INVALID_ARG;
+  }
+  int dev;
+  unsigned int* err;
+  if ((s = device_setup(&dev, &err)) != LCSA_OK) return s;
+  PoolParams p{};
+  p.H = q->H;
+  p.Hb = q->Y / 8;
+  p.Wb = q->X / 8;
+  const lcsa_tensor* ts[2] = {q, k};
+  double* outs[2] = {q_pool, k_pool};
+  for (int i = 0; i < 2; ++i) {
+    PoolTensor& pt = p.t[i];
+    if (ts[i] == nullptr) { pt.units = 0; continue; }
+    pt.data = static_cast<const __nv_bfloat16*>(ts[i]->data);
+    pt.out = outs[i];
+    pt.sb = ts[i]->stride_b; pt.sh = ts[i]->stride_h; pt.st = ts[i]->stride_t;
+    pt.sy = ts[i]->stride_y; pt.sx = ts[i]->stride_x;
+    pt.T = ts[i]->T;
+    pt.nT = temporal_blocks(ts[i]->T);
+    pt.units = static_cast<int64_t>(ts[i]->B) * ts[i]->H * pt.nT * p.Hb * p.Wb;
+  }
+  const int64_t units = p.t[0].units + p.t[1].units;
+  const int64_t grid = (units + POOL_WARPS - 1) / POOL_WARPS;
+  if (grid > 0x7fffffff) return LCSA_ERR_SHAPE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (q->D == 128) pool_kernel<128><<<static_cast<unsigned>(grid), POOL_WARPS * 32, 0, cs>>>(p);
+  else pool_kernel<64><<<static_cast<unsigned>(grid), POOL_WARPS * 32, 0, cs>>>(p);
+  return launched();
+}
+
+lcsa_status lcsa_kv_append(lcsa_kv_cache* kv, const lcsa_tensor* k_new, const lcsa_tensor* v_new,
+                           const double* k_pool_new, int32_t stream_offset, lcsa_stream_t stream) {
+  lcsa_status s = check_cache(kv);
+  if (s != LCSA_OK) return s;
+  if ((s = check_tensor(k_new)) != LCSA_OK || (s = check_tensor(v_new)) != LCSA_OK) return s;
+  if (k_pool_new == nullptr) return LCSA_ERR_INVALID_ARG;
+  if (!aligned16(k_pool_new)) return LCSA_ERR_ALIGN;
+  const lcsa_tensor* kn = k_new;
+  if (v_new->B != kn->B || v_new->H != kn->H || v_new->T != kn->T || v_new->Y != kn->Y ||
+      v_new->X != kn->X || v_new->D != kn->D)
+    return LCSA_ERR_SHAPE;
+  if (kn->H != kv->H || kn->Y != kv->Y || kn->X != kv->X || kn->D != kv->D) return LCSA_ERR_SHAPE;
+  if (stream_offset < 0 || stream_offset + kn->B > kv->B) return LCSA_ERR_INVALID_ARG;
+  const int Tn = kn->T;
+  const int cap = kv->cap_frames;
+  AppendParams p{};
+  int64_t new_begin[LCSA_MAX_STREAMS], new_end[LCSA_MAX_STREAMS];
+  for (int bn = 0; bn < kn->B; ++bn) {
+    const int b = bn + stream_offset;
+    const bool empty = kv->end[b] == kv->begin[b];
+    if (!empty && (Tn & 1)) return LCSA_ERR_SHAPE;  // odd chunks only start a stream
+    const int64_t first = empty ? kv->end[b] + (Tn & 1) : kv->end[b];
+    const int64_t e = first + Tn;
+    const int64_t old_begin = empty ? first : kv->begin[b];
+    new_end[bn] = e;
+    new_begin[bn] = old_begin > e - cap ? old_begin : e - cap;
+    p.first_abs[bn] = first;
+  }
+  // Every stream of one call appends the same frames of the chunk: the newest
+  // min(Tn, cap) frames (cap is even, so the kept blocks are whole or the
+  // chunk's own one-frame oldest block).
+  const int f_first = Tn > cap ? Tn - cap : 0;
+  const int nTn = temporal_blocks(Tn);
+  const int copy_blocks = temporal_blocks(Tn - f_first);
+  int dev;
+  unsigned int* err;
+  if ((s = device_setup(&dev, &err)) != LCSA_OK) return s;
+  p.k_new = static_cast<const __nv_bfloat16*>(kn->data);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new->data);
+  p.kp_new = k_pool_new;
+  p.k_cache = static_cast<__nv_bfloat16*>(kv->k);
+  p.v_cache = static_cast<__nv_bfloat16*>(kv->v);
+  p.kp_cache = kv->k_pool;
+  p.ksb = kn->stride_b; p.ksh = kn->stride_h; p.kst = kn->stride_t; p.ksy = kn->stride_y; p.ksx = kn->stride_x;
+  p.vsb = v_new->stride_b; p.vsh = v_new->stride_h; p.vst = v_new->stride_t;
+  p.vsy = v_new->stride_y; p.vsx = v_new->stride_x;
+  p.Bn = kn->B; p.H = kn->H; p.Y = kn->Y; p.X = kn->X; p.D = kn->D;
+  p.Hb = kn->Y / 8; p.Wb = kn->X / 8;
+  p.cap = cap;
+  p.stream_offset = stream_offset;
+  p.f_first = f_first;
+  p.n_frames = Tn - f_first;
+  p.nTn = nTn;
+  p.tb_first = nTn - copy_blocks;
+  p.kv_planes = kn->B * kn->H * p.n_frames;
+  p.pool_planes = kn->B * kn->H * copy_blocks;
+  const int64_t planes = 2 * static_cast<int64_t>(p.kv_planes) + p.pool_planes;
+  if (planes > 65535) return LCSA_ERR_SHAPE;
+  const int64_t plane_vecs = static_cast<int64_t>(p.Y) * p.X * p.D / 8;
+  const int64_t gx = (plane_vecs + APPEND_CHUNK - 1) / APPEND_CHUNK;
+  kv_append_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(planes)), APPEND_THREADS, 0,
+                     static_cast<cudaStream_t>(stream)>>>(p);
+  if ((s = launched()) != LCSA_OK) return s;
+  for (int bn = 0; bn < kn->B; ++bn) {
+    kv->begin[bn + stream_offset] = new_begin[bn];
+    kv->end[bn + stream_offset] = new_end[bn];
+  }
+  return LCSA_OK;
+}
+
+int32_t lcsa_select_kmax(const lcsa_kv_cache* kv, int32_t q_frames, const lcsa_select_params* p) {
+  if (kv == nullptr || p == nullptr || q_frames < 1 || kv->B < 1 || kv->B > LCSA_MAX_STREAMS) return 0;
+  int nKT = 0;
+  for (int b = 0; b < kv->B; ++b) {
+    const int n = static_cast<int>((kv->end[b] >> 1) - (kv->begin[b] >> 1));
+    nKT = n > nKT ? n : nKT;
+  }
+  return kmax_for(nKT, temporal_blocks(q_frames), kv->Y / 8, kv->X / 8, p);
+}
+
+lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames, const lcsa_kv_cache* kv,
+                               const lcsa_select_params* sp, int32_t* blk_idx, int32_t* blk_cnt,
+                               lcsa_stream_t stream) {
+  lcsa_status s = check_cache(kv);
+  if (s != LCSA_OK) return s;
+  if (q_pool == nullptr || sp == nullptr || blk_idx == nullptr || blk_cnt == nullptr)
+    return LCSA_ERR_INVALID_ARG;
+  if (!aligned16(q_pool)) return LCSA_ERR_ALIGN;
+  if (sp->top_k < 0 || sp->kmax < 1 || !(sp->tie_eps >= 0.0)) return LCSA_ERR_INVALID_ARG;
+  if (sp->top_k == 0 && !(sp->density > 0.0 && sp->density <= 1.0)) return LCSA_ERR_INVALID_ARG;
+  if (sp->window < 0 || (sp->window > 0 && sp->window % 2 == 0)) return LCSA_ERR_INVALID_ARG;
+  if (sp->window_mode != LCSA_WINDOW_TRUNCATE && sp->window_mode != LCSA_WINDOW_PRESERVE)
+    return LCSA_ERR_INVALID_ARG;
+  if (q_frames < 1) return LCSA_ERR_SHAPE;
+  const int Hb = kv->Y / 8, Wb = kv->X / 8, HbWb = Hb * Wb;
+  const int nQT = temporal_blocks(q_frames);
+  int nKT_max = 0;
+  for (int b = 0; b < kv->B; ++b) {
+    if (kv->end[b] - kv->begin[b] < q_frames) return LCSA_ERR_SHAPE;  // queries are cached frames
+    const int n = static_cast<int>((kv->end[b] >> 1) - (kv->begin[b] >> 1));
+    nKT_max = n > nKT_max ? n : nKT_max;
+  }
+  if (kmax_for(nKT_max, nQT, Hb, Wb, sp) > sp->kmax) return LCSA_ERR_CAPACITY;
+  const int ncand_max = nKT_max * HbWb;
+  const int c_stride = ncand_max + 1;
+  const size_t smem = sizeof(double) * (static_cast<size_t>(SEL_ROWS) * kv->D +
+                                        static_cast<size_t>(SEL_TILE) * (kv->D + 1) +
+                                        static_cast<size_t>(SEL_ROWS) * c_stride);
+  if (smem > 227 * 1024) return LCSA_ERR_SHAPE;
+  int dev;
+  unsigned int* err;
+  if ((s = device_setup(&dev, &err)) != LCSA_OK) return s;
+  SelectParams p{};
+  p.q_pool = q_pool;
+  p.k_pool = kv->k_pool;
+  p.blk_idx = blk_idx;
+  p.blk_cnt = blk_cnt;
+  p.H = kv->H; p.D = kv->D; p.Hb = Hb; p.Wb = Wb; p.nQT = nQT;
+  p.cap_blk = kv->cap_frames / 2;
+  p.top_k = sp->top_k; p.window = sp->window; p.window_mode = sp->window_mode; p.kmax = sp->kmax;
+  p.c_stride = c_stride;
+  p.density = sp->density;
+  p.tie_eps = sp->tie_eps;
+  p.sqrt_d = std::sqrt(static_cast<double>(kv->D));
+  p.err = err;
+  for (int b = 0; b < kv->B; ++b) { p.kv_begin[b] = kv->begin[b]; p.kv_end[b] = kv->end[b]; }
+  const dim3 grid((HbWb + SEL_ROWS - 1) / SEL_ROWS, nQT, kv->B * kv->H);
+  select_kernel<<<grid, SEL_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  return launched();
+}
+
+lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_cache* kv, const int32_t* blk_idx,
+                                 const int32_t* blk_cnt, int32_t kmax, lcsa_tensor* o, float* lse,
+                                 lcsa_stream_t stream) {
+  lcsa_status s = check_tensor(q);
+  if (s != LCSA_OK) return s;
+  if ((s = check_cache(kv)) != LCSA_OK) return s;
+  if (o == nullptr) return LCSA_ERR_INVALID_ARG;
+  if ((s = check_tensor(o)) != LCSA_OK) return s;
+  if (blk_idx == nullptr || blk_cnt == nullptr || kmax < 1) return LCSA_ERR_INVALID_ARG;
+  if (q->B != kv->B || q->H != kv->H || q->Y != kv->Y || q->X != kv->X || q->D != kv->D)
+    return LCSA_ERR_SHAPE;
+  if (o->B != q->B || o->H != q->H || o->T != q->T || o->Y != q->Y || o->X != q->X || o->D != q->D)
+    return LCSA_ERR_SHAPE;
+  for (int b = 0; b < kv->B; ++b)
+    if (kv->end[b] - kv->begin[b] < q->T) return LCSA_ERR_SHAPE;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LCSA_ERR_ALIGN;
+  int dev;
+  unsigned int* err;
+  if ((s = device_setup(&dev, &err)) != LCSA_OK) return s;
+  CUtensorMap tq, tk, tv;
+  const int64_t cs_x = kv->D, cs_y = static_cast<int64_t>(kv->X) * kv->D;
+  const int64_t cs_t = cs_y * kv->Y, cs_h = cs_t * kv->cap_frames;
+  if ((s = encode_map(&tq, q->data, q->B, q->H, q->T, q->Y, q->X, q->D, q->stride_h, q->stride_t,
+                      q->stride_y, q->stride_x)) != LCSA_OK ||
+      (s = encode_map(&tk, kv->k, kv->B, kv->H, kv->cap_frames, kv->Y, kv->X, kv->D, cs_h, cs_t, cs_y,
+                      cs_x)) != LCSA_OK ||
+      (s = encode_map(&tv, kv->v, kv->B, kv->H, kv->cap_frames, kv->Y, kv->X, kv->D, cs_h, cs_t, cs_y,
+                      cs_x)) != LCSA_OK)
+    return s;
+  AttnParams p{};
+  p.blk_idx = blk_idx;
+  p.blk_cnt = blk_cnt;
+  p.o = static_cast<__nv_bfloat16*>(o->data);
+  p.lse = lse;
+  p.osh = o->stride_h; p.ost = o->stride_t; p.osy = o->stride_y; p.osx = o->stride_x;
+  p.H = q->H; p.Tq = q->T; p.Y = q->Y; p.X = q->X; p.Hb = q->Y / 8; p.Wb = q->X / 8;
+  p.nQT = temporal_blocks(q->T);
+  p.nQB = p.nQT * p.Hb * p.Wb;
+  p.kmax = kmax;
+  p.cap = kv->cap_frames;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(q->D)));
+  p.wait_limit_ns = g_wait_limit_ns;
+  p.err = err;
+  for (int b = 0; b < kv->B; ++b) { p.kv_begin[b] = kv->begin[b]; p.kv_end[b] = kv->end[b]; }
+  const int64_t grid = static_cast<int64_t>(q->B) * q->H * p.nQB;
+  if (grid > 0x7fffffff) return LCSA_ERR_SHAPE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (q->D == 128)
+    attn_fwd_kernel<128><<<static_cast<unsigned>(grid), ATTN_THREADS, AttnLayout<128>::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+  else
+    attn_fwd_kernel<64><<<static_cast<unsigned>(grid), ATTN_THREADS, AttnLayout<64>::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+  return launched();
+}
+
+lcsa_status lcsa_last_device_error(lcsa_stream_t stream) {
+  int dev;
+  unsigned int* err;
+  lcsa_status s = device_setup(&dev, &err);
+  if (s != LCSA_OK) return s;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  unsigned int word = 0;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return LCSA_ERR_CUDA;
+  if (cudaMemcpyAsync(&word, err, sizeof(word), cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+      cudaMemsetAsync(err, 0, sizeof(word), cs) != cudaSuccess || cudaStreamSynchronize(cs) != cudaSuccess)
+    return LCSA_ERR_CUDA;
+  if (word & DEVERR_TIMEOUT) return LCSA_ERR_TIMEOUT;
+  if (word & DEVERR_BOUNDS) return LCSA_ERR_DEVICE_BOUNDS;
+  return LCSA_OK;
+}
+
+lcsa_status lcsa_debug_stalled_wait(uint64_t limit_ns, lcsa_stream_t stream) {
+  int dev;
+  unsigned int* err;
+  lcsa_status s = device_setup(&dev, &err);
+  if (s != LCSA_OK) return s;
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return LCSA_ERR_INVALID_ARG;
+  stalled_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, err);
+  return launched();
+}
+
+lcsa_status lcsa_debug_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns = ns == 0 ? kDefaultWaitNs : ns;
+  return LCSA_OK;
+}
+
+}  // extern "C"

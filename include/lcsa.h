@@ -1,0 +1,256 @@
+/*
+ * lcsa.h - C ABI of the B200 (sm_100a) locality-constrained block-sparse
+ * causal attention library (liblcsa.so).
+ *
+ * The method is FlashVSR's sparse attention ("FlashVSR: Towards Real-time
+ * Diffusion-Based Streaming Video Super-Resolution"; fmread summary of the
+ * paper, section 2.2 "stage 2: block-sparse causal attention adaptation",
+ * section 2.2 "stage 3" for the KV cache, section 2.3 "locality-constrained
+ * sparse attention"). One streaming step is four calls, all asynchronous on
+ * the caller's CUDA stream:
+ *
+ *   lcsa_pool_qk        mean-pool Q and K over 2x8x8 (t,y,x) token blocks
+ *   lcsa_kv_append      write the chunk's K, V and pooled K into the ring cache
+ *   lcsa_select_blocks  coarse block scores + causal/window masks + top-K
+ *   lcsa_sparse_attn_fwd  online-softmax attention over the kept blocks
+ *
+ * Conventions
+ * - Memory: the caller owns every buffer. The library allocates no device or
+ *   host memory (the attention kernel allocates tensor memory on the SM for
+ *   its own lifetime only). A call writes only its output arguments.
+ * - Pointers named "device" must be CUDA device pointers on the current
+ *   device; all others are host pointers.
+ * - Errors: argument and shape errors are returned synchronously, before any
+ *   launch, and leave every output untouched. Errors detected inside a kernel
+ *   (a wait that timed out, an index out of range) are recorded in a
+ *   per-device error word that lcsa_last_device_error() reads and clears;
+ *   kernels never trap.
+ * - Element types: Q, K, V, O are bf16 (raw 16-bit storage); pooled features
+ *   and block scores are float64; LSE is float32; block ids are int32.
+ * - Token tensors use lcsa_tensor: extents [B][H][T][Y][X][D], D unit stride,
+ *   element strides for B, H, T, Y, X. Requirements: D is 64 or 128; Y and X
+ *   multiples of 8; data 16-byte aligned; every stride a multiple of 8
+ *   elements; stride_b == H * stride_h (batch and heads must merge).
+ * - Blocks: 2 (t) x 8 (y) x 8 (x) = 128 tokens. In time, blocks are counted
+ *   backwards from the newest frame, so a tensor with an odd frame count has
+ *   a one-frame (64-token) OLDEST block. Block id within a frame sequence:
+ *   t_blk * Hb * Wb + y_blk * Wb + x_blk, t_blk oldest first, Hb = Y/8,
+ *   Wb = X/8.
+ */
+#ifndef LCSA_H
+#define LCSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LCSA_API __attribute__((visibility("default")))
+#else
+#define LCSA_API
+#endif
+
+#define LCSA_ABI_VERSION 1
+#define LCSA_MAX_STREAMS 64
+
+/* A cudaStream_t passed through as an opaque handle (NULL = default stream). */
+typedef void* lcsa_stream_t;
+
+typedef enum lcsa_status {
+  LCSA_OK = 0,
+  LCSA_ERR_INVALID_ARG = -1,  /* null pointer, bad enum, bad parameter value  */
+  LCSA_ERR_SHAPE = -2,        /* extents inconsistent or unsupported           */
+  LCSA_ERR_ALIGN = -3,        /* pointer or stride misaligned                  */
+  LCSA_ERR_CAPACITY = -4,     /* KV cache or blk_idx row capacity exceeded     */
+  LCSA_ERR_WORKSPACE = -5,    /* reserved                                      */
+  LCSA_ERR_CUDA = -6,         /* a CUDA runtime/driver call failed             */
+  LCSA_ERR_TIMEOUT = -7,      /* a kernel wait gave up (device error word)     */
+  LCSA_ERR_DEVICE_BOUNDS = -8 /* a kernel saw an out-of-range block id         */
+} lcsa_status;
+
+enum { LCSA_WINDOW_TRUNCATE = 0, LCSA_WINDOW_PRESERVE = 1 };
+
+/* A token tensor [B][H][T][Y][X][D] of bf16 in device memory. */
+typedef struct lcsa_tensor {
+  void* data;  /* device */
+  int32_t B, H, T, Y, X, D;
+  int64_t stride_b, stride_h, stride_t, stride_y, stride_x; /* in elements */
+} lcsa_tensor;
+
+/*
+ * Streaming KV cache of B streams (section 2.2, stage 3: later layers refine
+ * temporal consistency through a KV cache; section 3: 8-frame chunks).
+ *
+ * k, v    device, bf16, contiguous [B][H][cap_frames][Y][X][D]
+ * k_pool  device, float64, contiguous [B][H][cap_frames/2][Y/8][X/8][D]
+ * begin, end  host-side state of stream b: absolute indices of its oldest
+ *         valid frame and one past its newest; 0 <= end-begin <= cap_frames.
+ *         Absolute frame a lives in ring slot a % cap_frames; block m covers
+ *         absolute frames 2m and 2m+1 and its pooled K lives in slot
+ *         m % (cap_frames/2). end is kept even, so blocks never straddle a
+ *         chunk boundary; a stream whose first chunk has an odd number of
+ *         frames starts at an odd begin (its oldest block has one frame).
+ * cap_frames must be even. A fresh cache has begin[b] == end[b] == 0.
+ * The caller may also wrap plain K/V tensors of F frames (F even) as a cache
+ * with cap_frames = F, begin = 0, end = F and k_pool = their pooled K.
+ */
+typedef struct lcsa_kv_cache {
+  void* k;         /* device */
+  void* v;         /* device */
+  double* k_pool;  /* device */
+  int32_t B, H, cap_frames, Y, X, D;
+  int64_t begin[LCSA_MAX_STREAMS];
+  int64_t end[LCSA_MAX_STREAMS];
+} lcsa_kv_cache;
+
+/*
+ * Parameters of the block selection (section 2.2 stage 2: coarse block map
+ * and top-K; section 2.3: locality window with boundary-preserve or
+ * boundary-truncate rules).
+ *
+ * top_k     > 0: keep min(C_i, top_k) blocks per query block;
+ *           0: keep K_i = min(C_i, max(1, ceil(density * C_i))) where C_i is
+ *           the number of allowed (causal, in-window) key blocks of the row
+ *           and density * C_i is a float64 product.
+ * window    0: no window; else the odd side length of the square spatial
+ *           window in blocks (radius window/2), centred on the query block.
+ * window_mode  LCSA_WINDOW_TRUNCATE: clip the window at the frame edge;
+ *           LCSA_WINDOW_PRESERVE: shift it inward so it always spans
+ *           `window` blocks (start = max(0, min(y-r, Hb-window))).
+ * tie_eps   near-tie band (1e-5): with tau the K_i-th largest score, blocks
+ *           with score > tau+eps are kept and the remaining places go to the
+ *           lowest-index blocks with tau-eps <= score <= tau+eps.
+ * kmax      row capacity of blk_idx (>= every K_i; see lcsa_select_kmax).
+ */
+typedef struct lcsa_select_params {
+  int32_t top_k;
+  int32_t window;
+  int32_t window_mode;
+  int32_t kmax;
+  double density;
+  double tie_eps;
+} lcsa_select_params;
+
+/* ABI version of the loaded library (LCSA_ABI_VERSION). */
+LCSA_API int32_t lcsa_abi_version(void);
+
+/* Static description of a status code. */
+LCSA_API const char* lcsa_status_string(lcsa_status s);
+
+/*
+ * lcsa_pool_qk - block mean-pooling of Q and K (section 2.2, stage 2:
+ * "average pooling yields compact block-level features").
+ *
+ * q, k     token tensors (k may be NULL to pool Q only); their B, H, Y, X, D
+ *          must agree, T may differ.
+ * q_pool   device, float64, contiguous [B][H][ceil(Tq/2)][Y/8][X/8][D]
+ * k_pool   device, float64, contiguous [B][H][ceil(Tk/2)][Y/8][X/8][D]
+ *          (ignored when k is NULL).
+ * Each output is the arithmetic mean of the block's tokens (128, or 64 for a
+ * one-frame oldest block), accumulated in float64 (exact for bf16 inputs
+ * whose non-zero values in one block span at most 38 binades).
+ */
+LCSA_API lcsa_status lcsa_pool_qk(const lcsa_tensor* q, const lcsa_tensor* k,
+                         double* q_pool, double* k_pool, lcsa_stream_t stream);
+
+/*
+ * lcsa_kv_append - append a chunk to the streaming KV cache (section 2.2,
+ * stage 3 KV cache) and drop frames past the capacity.
+ *
+ * kv          cache (device buffers + host begin/end, updated on success).
+ * k_new, v_new  token tensors [Bn][H][Tn][Y][X][D] with the cache's H, Y, X,
+ *             D; they fill cache streams [stream_offset, stream_offset+Bn).
+ * k_pool_new  device, float64 [Bn][H][ceil(Tn/2)][Y/8][X/8][D], the pooled
+ *             K of the chunk (lcsa_pool_qk on k_new).
+ * Tn must be even, except for the first chunk of an empty stream, whose
+ * frames are then placed so that the oldest block holds one frame. Only the
+ * newest cap_frames frames of a chunk longer than the cache are written.
+ */
+LCSA_API lcsa_status lcsa_kv_append(lcsa_kv_cache* kv, const lcsa_tensor* k_new,
+                           const lcsa_tensor* v_new, const double* k_pool_new,
+                           int32_t stream_offset, lcsa_stream_t stream);
+
+/*
+ * Row capacity blk_idx needs for a selection with these parameters over the
+ * cache's current state and q_frames query frames (the largest K_i).
+ * Returns 0 on invalid arguments.
+ */
+LCSA_API int32_t lcsa_select_kmax(const lcsa_kv_cache* kv, int32_t q_frames,
+                         const lcsa_select_params* p);
+
+/*
+ * lcsa_select_blocks - coarse block map, masks and top-K (section 2.2,
+ * stage 2: "coarse block-to-block attention map ... keep only the most
+ * relevant top-K block pairs", causal masking; section 2.3 locality window).
+ *
+ * q_pool    device, float64 [B][H][ceil(q_frames/2)][Y/8][X/8][D]; the query
+ *           frames are the newest q_frames frames of every stream's cache.
+ * kv        cache whose k_pool holds the pooled keys; B, H, Y, X, D as q_pool.
+ * blk_idx   device, int32 [B][H][nQB][kmax]; row i receives the ids of its
+ *           kept key blocks in ascending order (id = t*Hb*Wb + y*Wb + x, t
+ *           counted from the stream's oldest cached block), unused tail
+ *           entries are -1.
+ * blk_cnt   device, int32 [B][H][nQB]; K_i per row.
+ * Scores are s_ij = (qbar_i . kbar_j) / sqrt(D) in float64, the dot product
+ * summed in channel order with every product rounded before it is added, so
+ * selections are reproducible bit for bit. Key block j is a candidate of
+ * query block i iff t_j <= t_i (block-level causality) and j lies in i's
+ * window.
+ */
+LCSA_API lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames,
+                               const lcsa_kv_cache* kv,
+                               const lcsa_select_params* p, int32_t* blk_idx,
+                               int32_t* blk_cnt, lcsa_stream_t stream);
+
+/*
+ * lcsa_sparse_attn_fwd - attention inside the kept blocks (section 2.2,
+ * stage 2: "apply full attention within the selected regions").
+ *
+ * q        token tensor [B][H][Tq][Y][X][D]: the newest Tq frames of each
+ *          stream of kv.
+ * kv       cache holding K and V (B, H, Y, X, D as q).
+ * blk_idx, blk_cnt, kmax  as written by lcsa_select_blocks (device).
+ * o        token tensor like q (bf16), device; receives
+ *          O_r = sum_t softmax_t(q_r . k_t / sqrt(D)) v_t over the tokens t of
+ *          the kept blocks of r's query block (a one-frame block contributes
+ *          its 64 tokens).
+ * lse      device, float32 contiguous [B][H][Tq][Y][X] natural-log
+ *          log-sum-exp of each row's scaled logits, or NULL.
+ * bf16 tensor-core products with float32 accumulation and softmax.
+ */
+LCSA_API lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_cache* kv,
+                                 const int32_t* blk_idx, const int32_t* blk_cnt,
+                                 int32_t kmax, lcsa_tensor* o, float* lse,
+                                 lcsa_stream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear the current device's error word.
+ * Returns LCSA_OK, LCSA_ERR_TIMEOUT or LCSA_ERR_DEVICE_BOUNDS (first set
+ * bit wins), or LCSA_ERR_CUDA if the synchronisation itself failed. The word
+ * is shared by every stream on the device.
+ */
+LCSA_API lcsa_status lcsa_last_device_error(lcsa_stream_t stream);
+
+/*
+ * Test hook: make the next kernel launches of the library on the current
+ * device see a wait limit of `ns` nanoseconds (0 restores the default of
+ * about one second). Used to exercise the timeout path without any fault.
+ */
+LCSA_API lcsa_status lcsa_debug_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Test hook: launch one thread that waits on a barrier nothing will ever
+ * arrive at, with a wait limit of `limit_ns` (1 ns .. 10 s). The wait gives up,
+ * the kernel records LCSA_ERR_TIMEOUT in the device error word and returns;
+ * the context stays usable. No fault, trap or hang is involved.
+ */
+LCSA_API lcsa_status lcsa_debug_stalled_wait(uint64_t limit_ns, lcsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LCSA_H */

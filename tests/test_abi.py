@@ -1,0 +1,95 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU and exports every
+entry point include/*.h declares; argument errors are returned before any
+CUDA call. No compute call is made here."""
+import ctypes as C
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_causal_lcsa_b200 import build as b
+    from block_sparse_causal_lcsa_b200 import _abi
+
+    b.build()
+    return _abi.load()
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names |= set(re.findall(r"LCSA_API\s+[\w\s\*]+?\b(lcsa_\w+)\s*\(", text))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    from block_sparse_causal_lcsa_b200 import _abi
+    assert names == set(_abi.PROTOTYPES), "ctypes prototypes out of sync with the header"
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.lcsa_abi_version() == 1
+    assert lib.lcsa_status_string(0) == b"ok"
+    assert b"timed out" in lib.lcsa_status_string(-7)
+
+
+def test_struct_layouts_match_header():
+    from block_sparse_causal_lcsa_b200 import _abi
+    # offsets computed from include/lcsa.h by hand (LP64)
+    assert C.sizeof(_abi.Tensor) == 8 + 6 * 4 + 5 * 8
+    assert _abi.Tensor.stride_b.offset == 32
+    assert C.sizeof(_abi.KVCacheStruct) == 3 * 8 + 6 * 4 + 2 * 64 * 8
+    assert _abi.KVCacheStruct.begin.offset == 48
+    assert C.sizeof(_abi.SelectParamsStruct) == 4 * 4 + 2 * 8
+
+
+def test_argument_errors_before_any_launch(lib):
+    from block_sparse_causal_lcsa_b200 import _abi
+    # null tensors / pointers are rejected before the device is touched
+    assert lib.lcsa_pool_qk(None, None, None, None, None) == _abi.ERR_INVALID_ARG
+    t = _abi.Tensor(0x1000, 1, 1, 2, 16, 16, 96, 0, 0, 0, 0, 0)
+    assert lib.lcsa_pool_qk(C.byref(t), None, 0x2000, None, None) == _abi.ERR_SHAPE  # D = 96
+    t.D = 128
+    t.stride_x, t.stride_y, t.stride_t, t.stride_h, t.stride_b = 128, 2048, 32768, 65536, 65536
+    t.data = 0x1008
+    assert lib.lcsa_pool_qk(C.byref(t), None, 0x2000, None, None) == _abi.ERR_ALIGN
+    t.data = 0x1000
+    t.stride_b = 3 * 65536  # batch and heads must merge
+    assert lib.lcsa_pool_qk(C.byref(t), None, 0x2000, None, None) == _abi.ERR_SHAPE
+    kv = _abi.KVCacheStruct()
+    assert lib.lcsa_kv_append(C.byref(kv), C.byref(t), C.byref(t), None, 0, None) == _abi.ERR_INVALID_ARG
+    kv.k, kv.v, kv.k_pool = 0x1000, 0x2000, 0x3000
+    kv.B, kv.H, kv.cap_frames, kv.Y, kv.X, kv.D = 1, 1, 5, 16, 16, 128
+    sp = _abi.SelectParamsStruct(2, 0, 0, 2, 0.0, 1e-5)
+    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, None) == _abi.ERR_SHAPE
+    kv.cap_frames = 6
+    kv.end[0] = 3  # end must stay even
+    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, None) == _abi.ERR_INVALID_ARG
+    kv.end[0] = 6
+    sp.window = 4  # even window
+    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, None) == _abi.ERR_INVALID_ARG
+    sp.window = 0
+    sp.kmax = 1  # K = 2 does not fit
+    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, None) == _abi.ERR_CAPACITY
+
+
+def test_select_kmax_host_rule(lib):
+    from block_sparse_causal_lcsa_b200 import _abi
+    kv = _abi.KVCacheStruct()
+    kv.B, kv.H, kv.cap_frames, kv.Y, kv.X, kv.D = 1, 12, 6, 48, 88, 128
+    kv.begin[0], kv.end[0] = 0, 6
+    sp = _abi.SelectParamsStruct(0, 0, 0, 0, 0.136, 1e-5)
+    assert lib.lcsa_select_kmax(C.byref(kv), 2, C.byref(sp)) == 27  # 198 candidates
+    kv.Y, kv.X = 96, 168
+    sp.window = 9
+    assert lib.lcsa_select_kmax(C.byref(kv), 2, C.byref(sp)) == 34  # 243 candidates

@@ -1,0 +1,254 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Pooled features and block selections must match bit for bit; attention output
+must be within max-abs 2e-2 and relative L2 1e-2 of the fp64 result (bf16
+inputs, fp32 accumulation). Small variants of every workload are compared on
+every row; the full-size workloads are compared on every selection row and on
+sampled query blocks of O.
+"""
+import numpy as np
+import pytest
+import torch
+
+import lcsa_inputs as li
+from oracle import lcsa_oracle as orc
+
+from lcsa_harness import (build_cache, check_output, check_selection, compare_all, oracle_head,
+                          params_of, ring_to_logical, run_gpu)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lc():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import block_sparse_causal_lcsa_b200 as m
+    return m
+
+
+SMALL = [
+    li.workload("tiny"),
+    li.small_variant(li.workload("chunk"), H=2, Y=24, X=40),
+    li.small_variant(li.workload("multistream"), H=2, Y=16, X=24),
+    li.small_variant(li.workload("uhr_truncate"), H=2, Y=48, X=56, window=3),
+    li.small_variant(li.workload("uhr_preserve"), H=2, Y=48, X=56, window=3),
+    li.small_variant(li.workload("clip_5"), H=1, Y=16, X=24),
+    li.small_variant(li.workload("clip"), H=1, Y=16, X=24),
+    li.small_variant(li.workload("clip_30"), H=1, Y=16, X=24),
+    li.small_variant(li.workload("tiny"), H=1, Y=16, X=16, D=128, kv_past=(4,), cap_frames=6),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_small_workloads_every_row(lc, w):
+    x = li.make_inputs(w)
+    g = run_gpu(lc, w, x)
+    assert g["err"] == 0
+    compare_all(w, x, g)
+
+
+FULL = ["chunk", "multistream", "uhr_truncate", "uhr_preserve"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_selection_all_rows_output_sampled(lc, name):
+    w = li.workload(name)
+    x = li.make_inputs(w)
+    g = run_gpu(lc, w, x)
+    assert g["err"] == 0
+    rng = np.random.default_rng(11)
+    nQB = g["blk_cnt"].shape[2]
+    rows = sorted(rng.choice(nQB, size=6, replace=False).tolist() + [0, nQB - 1])
+    heads = [0, w.H - 1]
+    for b in range(w.B):
+        for h in range(w.H):
+            sel_rows = None if h in heads else rows
+            ref = oracle_head(w, x, b, h, rows=rows if h in heads else [])
+            where = "%s b%d h%d" % (name, b, h)
+            assert np.array_equal(g["q_pool"][b, h].reshape(-1, w.D), ref["q_pool"]), where
+            assert np.array_equal(ring_to_logical(g["cache"], g["k_pool_ring"], b, h), ref["k_pool"]), where
+            check_selection(g["blk_idx"][b, h], g["blk_cnt"][b, h], ref["sel"], where)
+            if h in heads:
+                check_output(g["O"][b, h], ref["O"], g["LSE"][b, h], ref["LSE"], where)
+            del sel_rows
+
+
+def test_full_clip_selection_and_sampled_output(lc):
+    w = li.workload("clip")
+    x = li.make_inputs(w)
+    dev = "cuda"
+    k = x["k"][0].unsqueeze(0).to(dev)
+    v = x["v"][0].unsqueeze(0).to(dev)
+    q = x["q"].to(dev)
+    q_pool, k_pool = lc.pool_qk(q, k)
+    cache = lc.KVCache.wrap(k, v, k_pool)
+    params = params_of(lc, w)
+    idx, cnt = lc.select_blocks(q_pool, w.q_frames, cache, params)
+    o, lse = lc.sparse_attn_fwd(q, cache, idx, cnt)
+    torch.cuda.synchronize()
+    assert lc.last_device_error() == 0
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    O, L = o.double().cpu().numpy(), lse.double().cpu().numpy()
+    qp, kp = q_pool.cpu().numpy(), k_pool.cpu().numpy()
+    nQB = cnt.shape[2]
+    rows = [0, 65, 400, nQB - 66, nQB - 1]
+    for h in range(w.H):
+        qh, kh = orc.widen(x["q"][0, h]), orc.widen(x["k"][0][h])
+        rq, rk = orc.pool_blocks(qh), orc.pool_blocks(kh)
+        assert np.array_equal(qp[0, h].reshape(-1, w.D), rq) and np.array_equal(kp[0, h].reshape(-1, w.D), rk)
+        sel, Ks, Cs = orc.select_head(rq, rk, w.q_frames, w.q_frames, w.Y, w.X, density=w.density)
+        check_selection(idx[0, h], cnt[0, h], sel, "clip h%d" % h)
+        if h in (0, 7):
+            ro, rl = orc.attend_head(qh, kh, orc.widen(x["v"][0][h]), sel, rows)
+            check_output(O[0, h], ro, L[0, h], rl, "clip h%d" % h)
+
+
+def test_attention_on_oracle_mask(lc):
+    """O computed from the oracle's own block lists (selection errors excluded)."""
+    w = li.small_variant(li.workload("chunk"), H=2, Y=24, X=40)
+    x = li.make_inputs(w)
+    g = run_gpu(lc, w, x)
+    step = g["step"]
+    kmax = step.blk_idx.shape[-1]
+    idx = np.full(step.blk_idx.shape, -1, np.int32)
+    cnt = np.zeros(step.blk_cnt.shape, np.int32)
+    refs = {}
+    for h in range(w.H):
+        ref = oracle_head(w, x, 0, h)
+        refs[h] = ref
+        for i, s in enumerate(ref["sel"]):
+            s = s[::-1]  # any order of the kept blocks gives the same output
+            idx[0, h, i, :len(s)] = s
+            cnt[0, h, i] = len(s)
+    o, lse = lc.sparse_attn_fwd(g["q"], g["cache"], torch.from_numpy(idx).cuda(),
+                                torch.from_numpy(cnt).cuda())
+    torch.cuda.synchronize()
+    assert lc.last_device_error() == 0 and kmax == idx.shape[-1]
+    for h in range(w.H):
+        check_output(o[0, h].double().cpu().numpy(), refs[h]["O"], lse[0, h].double().cpu().numpy(),
+                     refs[h]["LSE"], "h%d" % h)
+
+
+def test_streaming_sequence_with_eviction(lc):
+    """Five 2-frame chunks through a 6-frame cache; every step against the
+    oracle applied to the concatenated, evicted timeline."""
+    w = li.Workload("stream", B=1, H=2, D=128, Y=16, X=24, q_frames=2, kv_past=(8,),
+                    cap_frames=6, density=0.4, seed=21)
+    x = li.make_inputs(w)
+    dev = "cuda"
+    cache = lc.KVCache(1, w.H, w.cap_frames, w.Y, w.X, w.D, device=dev)
+    step = lc.StreamingStep(cache, 2, params_of(lc, w))
+    F = x["k"][0].shape[1]
+    for s0 in range(0, F, 2):
+        kc = x["k"][0][:, s0:s0 + 2].unsqueeze(0).to(dev)
+        vc = x["v"][0][:, s0:s0 + 2].unsqueeze(0).to(dev)
+        qc = torch.randn((1, w.H, 2, w.Y, w.X, w.D), generator=torch.Generator().manual_seed(s0)).to(torch.bfloat16)
+        o, lse = step(qc.to(dev), kc, vc)
+        torch.cuda.synchronize()
+        assert lc.last_device_error() == 0
+        lo = max(0, s0 + 2 - w.cap_frames)
+        assert cache.state() == [(lo, s0 + 2)]
+        for h in range(w.H):
+            kt = orc.widen(x["k"][0][h, lo:s0 + 2])
+            vt = orc.widen(x["v"][0][h, lo:s0 + 2])
+            ref = orc.lcsa_head(orc.widen(qc[0, h]), kt, vt, density=w.density)
+            assert np.array_equal(ring_to_logical(cache, cache.k_pool.cpu().numpy(), 0, h), ref["k_pool"])
+            kc_ring = cache.k[0, h].cpu()
+            for f in range(lo, s0 + 2):
+                assert torch.equal(kc_ring[f % w.cap_frames], x["k"][0][h, f])
+            check_selection(step.blk_idx[0, h].cpu().numpy(), step.blk_cnt[0, h].cpu().numpy(), ref["sel"])
+            check_output(o[0, h].double().cpu().numpy(), ref["O"], lse[0, h].double().cpu().numpy(), ref["LSE"])
+
+
+@pytest.mark.parametrize("first,q_frames", [(1, 1), (3, 3), (5, 2)])
+def test_odd_first_chunk_partial_blocks(lc, first, q_frames):
+    """A stream whose first chunk has an odd frame count: the oldest key block
+    (and, for odd query counts, the oldest query block) holds one frame."""
+    w = li.Workload("odd", B=1, H=2, D=128, Y=16, X=16, q_frames=q_frames, kv_past=(first - q_frames,),
+                    cap_frames=8, density=0.5, seed=31 + first)
+    x = li.make_inputs(w)
+    dev = "cuda"
+    cache = lc.KVCache(1, w.H, w.cap_frames, w.Y, w.X, w.D, device=dev)
+    k = x["k"][0].unsqueeze(0).to(dev)
+    v = x["v"][0].unsqueeze(0).to(dev)
+    lc.kv_append(cache, k, v, lc.pool_qk(k)[0])
+    assert cache.state() == [(1, first + 1)]
+    q = x["q"].to(dev)
+    qp = lc.pool_qk(q)[0]
+    params = params_of(lc, w)
+    idx, cnt = lc.select_blocks(qp, q_frames, cache, params)
+    o, lse = lc.sparse_attn_fwd(q, cache, idx, cnt)
+    torch.cuda.synchronize()
+    assert lc.last_device_error() == 0
+    for h in range(w.H):
+        ref = oracle_head(w, x, 0, h)
+        assert np.array_equal(qp[0, h].reshape(-1, w.D).cpu().numpy(), ref["q_pool"])
+        assert np.array_equal(ring_to_logical(cache, cache.k_pool.cpu().numpy(), 0, h), ref["k_pool"])
+        check_selection(idx[0, h].cpu().numpy(), cnt[0, h].cpu().numpy(), ref["sel"])
+        check_output(o[0, h].double().cpu().numpy(), ref["O"], lse[0, h].double().cpu().numpy(), ref["LSE"])
+
+
+@pytest.mark.parametrize("kw", [dict(density=1.0), dict(top_k=1000), dict(top_k=1),
+                                dict(density=0.3, window=99, window_mode=1)])
+def test_degenerate_selection_parameters(lc, kw):
+    w = li.Workload("edge", B=1, H=1, D=128, Y=16, X=24, q_frames=2, kv_past=(4,), cap_frames=6,
+                    seed=41, **kw)
+    x = li.make_inputs(w)
+    g = run_gpu(lc, w, x)
+    assert g["err"] == 0
+    compare_all(w, x, g)
+
+
+def test_planted_ties_resolve_to_lowest_index(lc):
+    """Identical key blocks give exactly equal scores; the lowest ids win."""
+    w = li.Workload("ties", B=1, H=1, D=128, Y=16, X=16, q_frames=2, kv_past=(4,), cap_frames=6,
+                    top_k=3, seed=51)
+    x = li.make_inputs(w)
+    k = x["k"][0]
+    for t in (0, 2, 4):  # every temporal block a copy of the first one
+        k[:, t:t + 2] = k[:, 0:2]
+    g = run_gpu(lc, w, x)
+    compare_all(w, x, g)
+
+
+def test_argument_errors_leave_outputs_untouched(lc):
+    w = li.small_variant(li.workload("chunk"), H=1, Y=16, X=16)
+    x = li.make_inputs(w)
+    g = run_gpu(lc, w, x)
+    step = g["step"]
+    before = step.blk_idx.clone()
+    with pytest.raises(lc.LcsaError) as e:
+        lc.select_blocks(step.q_pool, 2, g["cache"], lc.SelectParams(density=0.5, window=4),
+                         step.kmax, step.blk_idx, step.blk_cnt)
+    assert e.value.status == -1
+    with pytest.raises(lc.LcsaError):
+        lc.select_blocks(step.q_pool, 2, g["cache"], lc.SelectParams(density=1.0), 1,
+                         step.blk_idx, step.blk_cnt)
+    torch.cuda.synchronize()
+    assert torch.equal(before, step.blk_idx)
+
+
+def test_wait_timeout_reports_and_context_survives(lc):
+    """A wait that nothing completes gives up after its limit (no fault, no
+    hang); the status reaches the host and the next calls still work."""
+    assert lc.last_device_error() == 0
+    lc.debug_stalled_wait(2_000_000)  # 2 ms
+    assert lc.last_device_error() == -7
+    assert lc.last_device_error() == 0  # cleared
+    w = li.workload("tiny")
+    x = li.make_inputs(w)
+    g = run_gpu(lc, w, x)
+    assert g["err"] == 0
+    compare_all(w, x, g)
+
+
+def test_out_of_range_block_id_is_reported(lc):
+    w = li.workload("tiny")
+    x = li.make_inputs(w)
+    g = run_gpu(lc, w, x)
+    step = g["step"]
+    bad = step.blk_idx.clone()
+    bad[0, 0, 0, 0] = 10_000
+    lc.sparse_attn_fwd(g["q"], g["cache"], bad, step.blk_cnt)
+    assert lc.last_device_error() == -8
