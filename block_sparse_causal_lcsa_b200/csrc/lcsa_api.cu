@@ -51,7 +51,9 @@ lcsa_status device_setup(int* dev_out, unsigned int** err_out) {
                              AttnLayout<128>::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnLayout<64>::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              227 * 1024) != cudaSuccess)
       return LCSA_ERR_CUDA;
     g_attr_done[dev] = true;
@@ -206,12 +208,11 @@ lcsa_status lcsa_pool_qk(const lcsa_tensor* q, const lcsa_tensor* k, double* q_p
     pt.nT = temporal_blocks(ts[i]->T);
     pt.units = static_cast<int64_t>(ts[i]->B) * ts[i]->H * pt.nT * p.Hb * p.Wb;
   }
-  const int64_t units = p.t[0].units + p.t[1].units;
-  const int64_t grid = (units + POOL_WARPS - 1) / POOL_WARPS;
+  const int64_t grid = p.t[0].units + p.t[1].units;  // one CTA per block
   if (grid > 0x7fffffff) return LCSA_ERR_SHAPE;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (q->D == 128) pool_kernel<128><<<static_cast<unsigned>(grid), POOL_WARPS * 32, 0, cs>>>(p);
-  else pool_kernel<64><<<static_cast<unsigned>(grid), POOL_WARPS * 32, 0, cs>>>(p);
+  if (q->D == 128) pool_kernel<128><<<static_cast<unsigned>(grid), POOL_THREADS, 0, cs>>>(p);
+  else pool_kernel<64><<<static_cast<unsigned>(grid), POOL_THREADS, 0, cs>>>(p);
   return launched();
 }
 
@@ -320,9 +321,7 @@ lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames, const lcs
   if (kmax_for(nKT_max, nQT, Hb, Wb, sp) > sp->kmax) return LCSA_ERR_CAPACITY;
   const int ncand_max = nKT_max * HbWb;
   const int c_stride = ncand_max + 1;
-  const size_t smem = sizeof(double) * (static_cast<size_t>(SEL_ROWS) * kv->D +
-                                        static_cast<size_t>(SEL_TILE) * (kv->D + 1) +
-                                        static_cast<size_t>(SEL_ROWS) * c_stride);
+  const size_t smem = select_smem_bytes(kv->D, c_stride);
   if (smem > 227 * 1024) return LCSA_ERR_SHAPE;
   int dev;
   unsigned int* err;
@@ -332,7 +331,7 @@ lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames, const lcs
   p.k_pool = kv->k_pool;
   p.blk_idx = blk_idx;
   p.blk_cnt = blk_cnt;
-  p.H = kv->H; p.D = kv->D; p.Hb = Hb; p.Wb = Wb; p.nQT = nQT;
+  p.H = kv->H; p.Hb = Hb; p.Wb = Wb; p.nQT = nQT;
   p.cap_blk = kv->cap_frames / 2;
   p.top_k = sp->top_k; p.window = sp->window; p.window_mode = sp->window_mode; p.kmax = sp->kmax;
   p.c_stride = c_stride;
@@ -342,7 +341,8 @@ lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames, const lcs
   p.err = err;
   for (int b = 0; b < kv->B; ++b) { p.kv_begin[b] = kv->begin[b]; p.kv_end[b] = kv->end[b]; }
   const dim3 grid((HbWb + SEL_ROWS - 1) / SEL_ROWS, nQT, kv->B * kv->H);
-  select_kernel<<<grid, SEL_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  if (kv->D == 128) select_kernel<128><<<grid, SEL_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  else select_kernel<64><<<grid, SEL_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
   return launched();
 }
 
