@@ -213,7 +213,7 @@ def run_ours(args, world, rank, local):
             if ev is not None:
                 ev[2].record()
             lc.select_blocks(step.q_pool, step.q_frames, step.cache, step.params, step.kmax,
-                             step.blk_idx, step.blk_cnt)
+                             step.blk_idx, step.blk_cnt, step.workspace)
             if ev is not None:
                 ev[3].record()
             lc.sparse_attn_fwd(q, step.cache, step.blk_idx, step.blk_cnt, step.o, step.lse)
@@ -238,6 +238,8 @@ def run_ours(args, world, rank, local):
         blk_cnt = torch.empty((1, w.H, nQB), dtype=torch.int32, device=dev)
         o = torch.empty_like(q)
         lse = torch.empty(q.shape[:5], dtype=torch.float32, device=dev)
+        sel_ws = torch.empty(max(lc.select_workspace_bytes(cache, w.q_frames), 16), dtype=torch.uint8,
+                             device=dev)
         base_state = cache.state()
 
         class _S:
@@ -251,7 +253,7 @@ def run_ours(args, world, rank, local):
             lc.pool_qk(q, k, q_pool, k_pool)
             if ev is not None:
                 ev[1].record()
-            lc.select_blocks(q_pool, w.q_frames, cache, params, kmax, blk_idx, blk_cnt)
+            lc.select_blocks(q_pool, w.q_frames, cache, params, kmax, blk_idx, blk_cnt, sel_ws)
             if ev is not None:
                 ev[2].record()
             lc.sparse_attn_fwd(q, cache, blk_idx, blk_cnt, o, lse)

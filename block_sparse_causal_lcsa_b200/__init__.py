@@ -12,6 +12,7 @@ from .api import (  # noqa: F401
     StreamingStep,
     WINDOW_PRESERVE,
     WINDOW_TRUNCATE,
+    debug_exp2_poly,
     debug_set_wait_limit_ns,
     debug_stalled_wait,
     kv_append,
@@ -19,6 +20,7 @@ from .api import (  # noqa: F401
     pool_qk,
     select_blocks,
     select_kmax,
+    select_workspace_bytes,
     sparse_attn_fwd,
     tensor_desc,
 )

@@ -64,22 +64,24 @@ PROTOTYPES = {
                                  C.c_void_p, C.c_int32, C.c_void_p]),
     "lcsa_select_kmax": (C.c_int32, [C.POINTER(KVCacheStruct), C.c_int32,
                                      C.POINTER(SelectParamsStruct)]),
+    "lcsa_select_workspace_bytes": (C.c_size_t, [C.POINTER(KVCacheStruct), C.c_int32]),
     "lcsa_select_blocks": (C.c_int, [C.c_void_p, C.c_int32, C.POINTER(KVCacheStruct),
                                      C.POINTER(SelectParamsStruct), C.c_void_p, C.c_void_p,
-                                     C.c_void_p]),
+                                     C.c_void_p, C.c_size_t, C.c_void_p]),
     "lcsa_sparse_attn_fwd": (C.c_int, [C.POINTER(Tensor), C.POINTER(KVCacheStruct), C.c_void_p,
                                        C.c_void_p, C.c_int32, C.POINTER(Tensor), C.c_void_p,
                                        C.c_void_p]),
     "lcsa_last_device_error": (C.c_int, [C.c_void_p]),
     "lcsa_debug_set_wait_limit_ns": (C.c_int, [C.c_uint64]),
     "lcsa_debug_stalled_wait": (C.c_int, [C.c_uint64, C.c_void_p]),
+    "lcsa_debug_exp2_poly": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p]),
 }
 
 
 def load(path: str = LIB_PATH) -> C.CDLL:
     if not os.path.exists(path):
         raise ImportError(
-            "liblcsa.so is not built (%s); run `python -m block_sparse_causal_lcsa_b200.build` "
+            "liblcsa.so is not built (%s); run `python block_sparse_causal_lcsa_b200/build.py` "
             "or __graft_entry__.build()" % path)
     lib = C.CDLL(path)
     for name, (res, args) in PROTOTYPES.items():

@@ -160,13 +160,20 @@ def select_kmax(cache: KVCache, q_frames: int, params: SelectParams) -> int:
     return int(_lib.lcsa_select_kmax(C.byref(cache.struct), q_frames, C.byref(sp)))
 
 
+def select_workspace_bytes(cache: KVCache, q_frames: int) -> int:
+    return int(_lib.lcsa_select_workspace_bytes(C.byref(cache.struct), q_frames))
+
+
 def select_blocks(q_pool: torch.Tensor, q_frames: int, cache: KVCache, params: SelectParams,
                   kmax: Optional[int] = None, blk_idx: Optional[torch.Tensor] = None,
-                  blk_cnt: Optional[torch.Tensor] = None,
+                  blk_cnt: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                   stream: Optional[torch.cuda.Stream] = None):
     """Top-K key blocks of every query block: (blk_idx [B,H,nQB,kmax], blk_cnt [B,H,nQB])."""
     if kmax is None:
         kmax = select_kmax(cache, q_frames, params)
+    need = select_workspace_bytes(cache, q_frames)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_pool.device)
     B, H, nQT, Hb, Wb, D = q_pool.shape
     if not q_pool.is_contiguous() or q_pool.dtype != torch.float64:
         raise ValueError("q_pool must be contiguous float64")
@@ -177,7 +184,8 @@ def select_blocks(q_pool: torch.Tensor, q_frames: int, cache: KVCache, params: S
         blk_cnt = torch.empty((B, H, nQB), dtype=torch.int32, device=q_pool.device)
     sp = params.struct(kmax)
     _check(_lib.lcsa_select_blocks(q_pool.data_ptr(), q_frames, C.byref(cache.struct), C.byref(sp),
-                                   blk_idx.data_ptr(), blk_cnt.data_ptr(), _stream(stream)),
+                                   blk_idx.data_ptr(), blk_cnt.data_ptr(), workspace.data_ptr(),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
            "lcsa_select_blocks")
     return blk_idx, blk_cnt
 
@@ -209,6 +217,16 @@ def debug_stalled_wait(limit_ns: int, stream: Optional[torch.cuda.Stream] = None
     _check(_lib.lcsa_debug_stalled_wait(limit_ns, _stream(stream)), "lcsa_debug_stalled_wait")
 
 
+def debug_exp2_poly(x: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """2^x through the attention kernel's FMA-pipe polynomial (test hook)."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("expected a contiguous CUDA float32 tensor")
+    y = torch.empty_like(x)
+    _check(_lib.lcsa_debug_exp2_poly(x.data_ptr(), y.data_ptr(), x.numel(), _stream(stream)),
+           "lcsa_debug_exp2_poly")
+    return y
+
+
 def debug_set_wait_limit_ns(ns: int) -> None:
     _check(_lib.lcsa_debug_set_wait_limit_ns(ns), "lcsa_debug_set_wait_limit_ns")
 
@@ -238,6 +256,8 @@ class StreamingStep:
             full.begin[b], full.end[b] = 0, cache.cap_frames
         sp = params.struct()
         self.kmax = int(_lib.lcsa_select_kmax(C.byref(full), q_frames, C.byref(sp)))
+        ws = int(_lib.lcsa_select_workspace_bytes(C.byref(full), q_frames))
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
         nQB = nQT * (Y // 8) * (X // 8)
         self.blk_idx = torch.empty((B, H, nQB, self.kmax), dtype=torch.int32, device=dev)
         self.blk_cnt = torch.empty((B, H, nQB), dtype=torch.int32, device=dev)
@@ -249,6 +269,6 @@ class StreamingStep:
         pool_qk(q, k_new, self.q_pool, self.k_pool, stream)
         kv_append(self.cache, k_new, v_new, self.k_pool, 0, stream)
         select_blocks(self.q_pool, self.q_frames, self.cache, self.params, self.kmax,
-                      self.blk_idx, self.blk_cnt, stream)
+                      self.blk_idx, self.blk_cnt, self.workspace, stream)
         sparse_attn_fwd(q, self.cache, self.blk_idx, self.blk_cnt, self.o, self.lse, stream=stream)
         return self.o, self.lse

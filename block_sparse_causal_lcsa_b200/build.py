@@ -1,6 +1,6 @@
 """Build liblcsa.so in-tree for sm_100a with nvcc.
 
-    python -m block_sparse_causal_lcsa_b200.build [--force]
+    python block_sparse_causal_lcsa_b200/build.py [--force] [-v]
 
 The library is one translation unit (``csrc/lcsa_api.cu`` includes the kernel
 headers) compiled with ``-gencode arch=compute_100a,code=sm_100a`` and linked

@@ -3,26 +3,36 @@
 // 5th-generation tensor cores of sm_100a.
 //
 // One CTA computes one 128-token query block of one (stream, head) against
-// its K_i kept key blocks, with an online softmax:
-//   warp 0      TMA producer: the Q tile once, then K and V tiles of each kept
-//               block into two 3-stage rings (5-D tensor maps over
-//               (d, x, y, frame, stream*head); one box = one frame of a block
-//               = 64 tokens x 64 channels, 128-byte swizzled). A K stage is
-//               released as soon as S_j has consumed it, a V stage once PV_j
-//               has, so loads run up to three blocks ahead.
-//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM
-//               accumulators (128 lanes x 128 fp32 columns), then
-//               O += P_j V_j with P_j read from tensor memory and V_j from
-//               shared memory. S_{j+1} is issued before PV_j, so the tensor
-//               core computes the next scores while the softmax runs.
+// its K_i kept key blocks, with an online softmax. Seven warps:
+//   warps 0, 6  TMA producers: warp 0 loads the Q tile once and the K tile of
+//               each kept block, warp 6 the V tiles, into two 3-stage rings
+//               (5-D tensor maps over (d, x, y, frame, stream*head); one box =
+//               one frame of a block = 64 tokens x 64 channels, 128-byte
+//               swizzled). A K stage is released as soon as S_j has consumed
+//               it, a V stage once PV_j has; separate producers let the K
+//               loads run ahead of the V stages the softmax holds up.
+//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into one of THREE TMEM
+//               score buffers (128 lanes x 128 fp32 columns each), then
+//               O += P_j V_j with P_j read from tensor memory. Scores run up to
+//               two blocks ahead of the softmax (S_{j+2} is issued right after
+//               PV_j), so neither side waits for the other in steady state.
+//               Before an S MMA reuses the buffer a PV MMA read P from, the
+//               issuer waits for that PV to complete: MMAs into different
+//               accumulators are not ordered with respect to each other.
 //   warps 2-5   softmax warpgroup, one query row per thread (= TMEM lane):
 //               tcgen05.ld of S_j, mask the missing frame of a one-frame
 //               block, running max with lazy rescaling of O (only when the
-//               max grows by more than 2^8), P = 2^(s*log2e/sqrt(d) - m) on
-//               the special-function unit, rounded to bf16 and stored with
-//               tcgen05.st over the first 64 columns of S_j; row sums in
-//               fp32; at the end O / l to bf16 and the log-sum-exp.
-// Tensor memory: 512 columns (S0 | S1 | O). Shared memory for D = 128:
+//               max grows by more than 2^8), P = 2^(s*log2e/sqrt(d) - m) with
+//               packed fp32x2 arithmetic - exponentials on the
+//               special-function unit (every EXP_POLY_EVERY-th pair could go
+//               to a polynomial on the FMA pipe; measured slower here, so
+//               none does) - rounded to bf16 with integer ops
+//               (the special-function pipe also runs float->bf16
+//               conversions, so they would compete with the exponentials) and
+//               stored with tcgen05.st over the first 64 columns of S_j's
+//               buffer; row sums in fp32; at the end O / l in bf16 and the
+//               log-sum-exp.
+// Tensor memory: 512 columns (S0 | S1 | S2 | O). Shared memory for D = 128:
 // Q 32 KB + K 3x32 KB + V 3x32 KB = 224 KB, one CTA per SM.
 // Every wait is bounded; on a timeout the CTA drains its in-flight copies and
 // MMAs, frees its tensor memory and exits with the error word set.
@@ -32,7 +42,10 @@
 
 namespace lcsa {
 
-constexpr int KV_STAGES = 3;
+constexpr int K_STAGES = 3;
+constexpr int V_STAGES = 3;
+constexpr int S_BUFS = 3;
+constexpr int EXP_POLY_EVERY = 1 << 30;   // exponent pairs sent to the FMA-pipe polynomial (none)
 
 template <int D>
 struct AttnLayout {
@@ -41,8 +54,8 @@ struct AttnLayout {
   static constexpr int BOX_BYTES = 64 * 128;       // one frame of a block, 64 channels
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + TILE_BYTES;
-  static constexpr int OFF_V = OFF_K + KV_STAGES * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_V + KV_STAGES * TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + K_STAGES * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_V + V_STAGES * TILE_BYTES;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
 };
@@ -50,20 +63,21 @@ struct AttnLayout {
 // mbarrier slots
 enum : int {
   B_Q_FULL = 0,
-  B_K_FULL = 1,                        // KV_STAGES
-  B_K_EMPTY = B_K_FULL + KV_STAGES,    // KV_STAGES
-  B_V_FULL = B_K_EMPTY + KV_STAGES,    // KV_STAGES
-  B_V_EMPTY = B_V_FULL + KV_STAGES,    // KV_STAGES
-  B_S_FULL = B_V_EMPTY + KV_STAGES,    // 2 TMEM buffers
-  B_P_FULL = B_S_FULL + 2,             // 2
-  B_PV_DONE = B_P_FULL + 2,            // 2
+  B_K_FULL = 1,                        // K_STAGES
+  B_K_EMPTY = B_K_FULL + K_STAGES,     // K_STAGES
+  B_V_FULL = B_K_EMPTY + K_STAGES,     // V_STAGES
+  B_V_EMPTY = B_V_FULL + V_STAGES,     // V_STAGES
+  B_S_FULL = B_V_EMPTY + V_STAGES,     // S_BUFS
+  B_P_FULL = B_S_FULL + S_BUFS,        // S_BUFS (128 softmax arrivals)
+  B_PV_DONE = B_P_FULL + S_BUFS,       // 2, by parity of the block index
   B_DRAIN = B_PV_DONE + 2,
   B_COUNT = B_DRAIN + 1
 };
 
-constexpr int ATTN_THREADS = 192;
+constexpr int ATTN_THREADS = 224;
+constexpr int SOFTMAX_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_O_COL = 256;
+constexpr uint32_t TMEM_O_COL = 128 * S_BUFS;
 
 struct AttnParams {
   const int32_t* blk_idx;    // [B*H][nQB][kmax]
@@ -93,7 +107,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T: A (M x 16, bf16 pairs per 32-bit column)
+// D[tmem] (+)= A[tmem] * B[smem]^T: A (128 x 16, bf16 pairs per 32-bit column)
 // from tensor memory, one 128xNx16 step issued by one thread.
 __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                         uint32_t idesc, uint32_t accumulate) {
@@ -145,7 +159,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i)
-      mbar_init(bar(i), (i == B_P_FULL || i == B_P_FULL + 1) ? 128u : 1u);
+      mbar_init(bar(i), (i >= B_P_FULL && i < B_P_FULL + S_BUFS) ? SOFTMAX_THREADS : 1u);
     *abort_flag = 0;
     mbar_init_fence();
     tma_prefetch_map(&tmQ);
@@ -169,49 +183,72 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     return blk;
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0 && n > 0) {
-      auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar_full, int x8, int y8,
-                           int fr0, int fr1) {
+  // One 128-token tile = 2 frames x D/64 channel columns of 8 KB boxes.
+  auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar_full, int x8, int y8,
+                       int fr0, int fr1) {
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_5d(dst + c * L::CHUNK_BYTES, map, bar_full, c * 64, x8, y8, fr0, bh);
-          tma_load_5d(dst + c * L::CHUNK_BYTES + L::BOX_BYTES, map, bar_full, c * 64, x8, y8, fr1, bh);
-        }
-      };
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_5d(dst + c * L::CHUNK_BYTES, map, bar_full, c * 64, x8, y8, fr0, bh);
+      tma_load_5d(dst + c * L::CHUNK_BYTES + L::BOX_BYTES, map, bar_full, c * 64, x8, y8, fr1, bh);
+    }
+  };
+  // Ring slots of a key block's two frames; a one-frame block loads its frame twice.
+  auto tile_coords = [&](int blk, int& x8, int& y8, int& s0, int& s1) {
+    const int tk = blk / HbWb, spk = blk % HbWb;
+    const int64_t m = m_first + tk;
+    const int64_t a1 = 2 * m + 1;
+    const int64_t a0 = (2 * m < begin) ? a1 : 2 * m;
+    s0 = static_cast<int>(a0 % p.cap);
+    s1 = static_cast<int>(a1 % p.cap);
+    x8 = 8 * (spk % p.Wb);
+    y8 = 8 * (spk / p.Wb);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ Q + K producer
+    if (lane == 0 && n > 0) {
       mbar_arrive_expect_tx(bar(B_Q_FULL), L::TILE_BYTES);
       // a missing older query frame is replaced by the newer one (rows not stored)
       load_tile(&tmQ, sbase + L::OFF_Q, bar(B_Q_FULL), 8 * xq, 8 * yq, fq0 < 0 ? fq0 + 1 : fq0, fq0 + 1);
-      int issued_k = 0, issued_v = 0;
+      int issued_k = 0;
       int next_blk = checked(blist[0]);
       for (int j = 0; j < n; ++j) {
         const int blk = next_blk;
         if (j + 1 < n) next_blk = checked(blist[j + 1]);
-        const int st = j % KV_STAGES;
-        const uint32_t ph = ((j / KV_STAGES) - 1) & 1;
-        const int tk = blk / HbWb, spk = blk % HbWb;
-        const int64_t m = m_first + tk;
-        const int64_t a1 = 2 * m + 1;
-        const int64_t a0 = (2 * m < begin) ? a1 : 2 * m;   // one-frame block: load its frame twice
-        const int s0 = static_cast<int>(a0 % p.cap), s1 = static_cast<int>(a1 % p.cap);
-        const int x8 = 8 * (spk % p.Wb), y8 = 8 * (spk / p.Wb);
-        if (j >= KV_STAGES && !wait_bounded(bar(B_K_EMPTY + st), ph, w)) break;
-        mbar_arrive_expect_tx(bar(B_K_FULL + st), L::TILE_BYTES);
-        load_tile(&tmK, sbase + L::OFF_K + st * L::TILE_BYTES, bar(B_K_FULL + st), x8, y8, s0, s1);
+        int x8, y8, s0, s1;
+        tile_coords(blk, x8, y8, s0, s1);
+        const int ks = j % K_STAGES;
+        if (j >= K_STAGES && !wait_bounded(bar(B_K_EMPTY + ks), ((j / K_STAGES) - 1) & 1, w)) break;
+        mbar_arrive_expect_tx(bar(B_K_FULL + ks), L::TILE_BYTES);
+        load_tile(&tmK, sbase + L::OFF_K + ks * L::TILE_BYTES, bar(B_K_FULL + ks), x8, y8, s0, s1);
         issued_k = j + 1;
-        if (j >= KV_STAGES && !wait_bounded(bar(B_V_EMPTY + st), ph, w)) break;
-        mbar_arrive_expect_tx(bar(B_V_FULL + st), L::TILE_BYTES);
-        load_tile(&tmV, sbase + L::OFF_V + st * L::TILE_BYTES, bar(B_V_FULL + st), x8, y8, s0, s1);
-        issued_v = j + 1;
       }
       if (*abort_flag) {
         // let the copies already in flight land before the CTA goes away
         drain_wait(bar(B_Q_FULL), 0, w.limit_ns);
-        for (int j = issued_k > KV_STAGES ? issued_k - KV_STAGES : 0; j < issued_k; ++j)
-          drain_wait(bar(B_K_FULL + j % KV_STAGES), (j / KV_STAGES) & 1, w.limit_ns);
-        for (int j = issued_v > KV_STAGES ? issued_v - KV_STAGES : 0; j < issued_v; ++j)
-          drain_wait(bar(B_V_FULL + j % KV_STAGES), (j / KV_STAGES) & 1, w.limit_ns);
+        for (int j = issued_k > K_STAGES ? issued_k - K_STAGES : 0; j < issued_k; ++j)
+          drain_wait(bar(B_K_FULL + j % K_STAGES), (j / K_STAGES) & 1, w.limit_ns);
+      }
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ V producer
+    if (lane == 0 && n > 0) {
+      int issued_v = 0;
+      int next_blk = checked(blist[0]);
+      for (int j = 0; j < n; ++j) {
+        const int blk = next_blk;
+        if (j + 1 < n) next_blk = checked(blist[j + 1]);
+        int x8, y8, s0, s1;
+        tile_coords(blk, x8, y8, s0, s1);
+        const int vs = j % V_STAGES;
+        if (j >= V_STAGES && !wait_bounded(bar(B_V_EMPTY + vs), ((j / V_STAGES) - 1) & 1, w)) break;
+        mbar_arrive_expect_tx(bar(B_V_FULL + vs), L::TILE_BYTES);
+        load_tile(&tmV, sbase + L::OFF_V + vs * L::TILE_BYTES, bar(B_V_FULL + vs), x8, y8, s0, s1);
+        issued_v = j + 1;
+      }
+      if (*abort_flag) {
+        for (int j = issued_v > V_STAGES ? issued_v - V_STAGES : 0; j < issued_v; ++j)
+          drain_wait(bar(B_V_FULL + j % V_STAGES), (j / V_STAGES) & 1, w.limit_ns);
       }
     }
   } else if (warp == 1) {
@@ -220,8 +257,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       constexpr uint32_t ID_S = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, true);
       auto issue_s = [&](int j) -> bool {
-        const int ks = j % KV_STAGES;
-        if (!wait_bounded(bar(B_K_FULL + ks), (j / KV_STAGES) & 1, w)) return false;
+        const int ks = j % K_STAGES;
+        if (!wait_bounded(bar(B_K_FULL + ks), (j / K_STAGES) & 1, w)) return false;
         tc_fence_after();
         const uint32_t qa = sbase + L::OFF_Q;
         const uint32_t ka = sbase + L::OFF_K + ks * L::TILE_BYTES;
@@ -229,10 +266,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int kk = 0; kk < D / 16; ++kk) {
           // K-major operands: 16 channels = 32 bytes inside a 128-byte swizzled row
           const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + (j & 1) * 128, desc_sw128(qa + off, 16, 1024),
+          umma_ss(tmem + (j % S_BUFS) * 128, desc_sw128(qa + off, 16, 1024),
                   desc_sw128(ka + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
         }
-        umma_commit(bar(B_S_FULL + (j & 1)));
+        umma_commit(bar(B_S_FULL + j % S_BUFS));
         umma_commit(bar(B_K_EMPTY + ks));
         return true;
       };
@@ -240,15 +277,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (ok) {
         tc_fence_after();
         ok = issue_s(0);
+        if (ok && n > 1) ok = issue_s(1);
       }
       for (int j = 0; ok && j < n; ++j) {
-        const int sb = j & 1;
-        const int vs = j % KV_STAGES;
-        // S_{j+1} overwrites the TMEM buffer of P_{j-1}; PV_{j-1} was issued
-        // before it and tcgen05 MMAs of one thread execute in order.
-        if (j + 1 < n && !(ok = issue_s(j + 1))) break;
-        if (!(ok = wait_bounded(bar(B_P_FULL + sb), (j >> 1) & 1, w))) break;
-        if (!(ok = wait_bounded(bar(B_V_FULL + vs), (j / KV_STAGES) & 1, w))) break;
+        const int sb = j % S_BUFS;
+        const int vs = j % V_STAGES;
+        if (!(ok = wait_bounded(bar(B_P_FULL + sb), (j / S_BUFS) & 1, w))) break;
+        if (!(ok = wait_bounded(bar(B_V_FULL + vs), (j / V_STAGES) & 1, w))) break;
         tc_fence_after();
         const uint32_t va = sbase + L::OFF_V + vs * L::TILE_BYTES;
 #pragma unroll
@@ -260,8 +295,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                   desc_sw128(va + kk * 2048, L::CHUNK_BYTES, 1024), ID_PV,
                   (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(bar(B_PV_DONE + sb));
+        umma_commit(bar(B_PV_DONE + (j & 1)));
         umma_commit(bar(B_V_EMPTY + vs));
+        if (j + 2 < n) {
+          // S_{j+2} overwrites the buffer PV_{j-1} read P_{j-1} from. MMAs into
+          // different accumulators are not ordered, so wait until PV_{j-1}
+          // has completed (normally long done: PV_j was queued behind it).
+          if (j >= 1 && !(ok = wait_bounded(bar(B_PV_DONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, w))) break;
+          if (!(ok = issue_s(j + 2))) break;
+        }
       }
       // no MMA may still be running when the tensor memory is released
       umma_commit(bar(B_DRAIN));
@@ -274,14 +316,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const bool oldest_partial = (begin & 1) != 0; // the oldest cached block has one frame
     const float scale = p.scale_log2;
+    const uint64_t sc2 = f2_pack(scale, scale);
     float m_run = -INFINITY, l_run = 0.f;         // running max (log2 units) and sum
     bool done = n > 0;
     int next_blk = n > 0 ? checked(blist[0]) : 0;
     for (int j = 0; j < n; ++j) {
-      const int sb = j & 1;
+      const int sb = j % S_BUFS;
       const bool partial = oldest_partial && next_blk < HbWb;
       if (j + 1 < n) next_blk = checked(blist[j + 1]);
-      if (!warp_wait(bar(B_S_FULL + sb), (j >> 1) & 1, w)) { done = false; break; }
+      if (!warp_wait(bar(B_S_FULL + sb), (j / S_BUFS) & 1, w)) { done = false; break; }
       tc_fence_after();
       uint32_t s[128];
       tmem_ld_32x32b_x32(t_lane + sb * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
@@ -293,13 +336,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = __float_as_uint(-INFINITY);
       }
-      float mx0 = -INFINITY, mx1 = -INFINITY;
+      float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        mx0 = fmaxf(mx0, __uint_as_float(s[c]));
-        mx1 = fmaxf(mx1, __uint_as_float(s[c + 1]));
+      for (int c = 0; c < 128; c += 8) {
+        a0 = fmax3(a0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        a1 = fmax3(a1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+        a2 = fmax3(a2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+        a3 = fmax3(a3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
       }
-      const float mx = fmaxf(mx0, mx1) * scale;   // scale > 0: max commutes with it
+      const float mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * scale;  // scale > 0
       float m_new = m_run;
       if (j == 0 || mx > m_run + 8.f) m_new = mx;
       if (j > 0 && __any_sync(0xffffffffu, m_new != m_run)) {
@@ -320,23 +365,32 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         l_run *= alpha;
       }
       m_run = m_new;
-      const float neg_m = -m_run;
+      const uint64_t nm2 = f2_pack(-m_run, -m_run);
+      uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = f2_pack(0.f, 0.f);
       uint32_t pk[64];
-      float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * c]), scale, neg_m));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * c + 1]), scale, neg_m));
-        const float p2 = ex2_approx(fmaf(__uint_as_float(s[2 * c + 2]), scale, neg_m));
-        const float p3 = ex2_approx(fmaf(__uint_as_float(s[2 * c + 3]), scale, neg_m));
-        sum0 += p0;
-        sum1 += p1;
-        sum2 += p2;
-        sum3 += p3;
-        pk[c] = pack_bf16x2(p0, p1);
-        pk[c + 1] = pack_bf16x2(p2, p3);
+      for (int c = 0; c < 64; ++c) {
+        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sc2, nm2);
+        uint64_t e2;
+        if ((c % EXP_POLY_EVERY) == EXP_POLY_EVERY - 1) {
+          e2 = exp2_poly_f2(x2);
+        } else {
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        }
+        if (c & 1) acc1 = f2_add(acc1, e2);
+        else acc0 = f2_add(acc0, e2);
+        float e0, e1;
+        f2_unpack(e2, e0, e1);
+        pk[c] = pack_bf16x2_pos(e0, e1);
       }
-      l_run += (sum0 + sum1) + (sum2 + sum3);
+      {
+        float s0, s1, s2, s3;
+        f2_unpack(acc0, s0, s1);
+        f2_unpack(acc1, s2, s3);
+        l_run += (s0 + s1) + (s2 + s3);
+      }
       // P_j over the first 64 columns of S_j's buffer (S_j has been read)
       tmem_st_32x32b_x32(t_lane + sb * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
       tmem_st_32x32b_x32(t_lane + sb * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));

@@ -51,10 +51,10 @@ lcsa_status device_setup(int* dev_out, unsigned int** err_out) {
                              AttnLayout<128>::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnLayout<64>::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             227 * 1024) != cudaSuccess ||
-        cudaFuncSetAttribute(select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             227 * 1024) != cudaSuccess)
+        cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(score_smem_bytes(128))) != cudaSuccess ||
+        cudaFuncSetAttribute(score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(score_smem_bytes(64))) != cudaSuccess)
       return LCSA_ERR_CUDA;
     g_attr_done[dev] = true;
   }
@@ -134,6 +134,21 @@ __global__ void stalled_wait_kernel(uint64_t limit_ns, unsigned int* err) {
     mbar_init_fence();
     const WaitCtx w{limit_ns, &abort_flag, err};
     wait_bounded(smem_u32(&bar), 0, w);
+  }
+}
+
+// Evaluates the attention kernel's FMA-pipe 2^x polynomial elementwise.
+__global__ void exp2_poly_kernel(const float* x, float* y, int64_t n) {
+  const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    float a, b;
+    f2_unpack(exp2_poly_f2(f2_pack(x[i], x[i + 1])), a, b);
+    y[i] = a;
+    y[i + 1] = b;
+  } else if (i < n) {
+    float a, b;
+    f2_unpack(exp2_poly_f2(f2_pack(x[i], 0.f)), a, b);
+    y[i] = a;
   }
 }
 
@@ -296,14 +311,32 @@ int32_t lcsa_select_kmax(const lcsa_kv_cache* kv, int32_t q_frames, const lcsa_s
   return kmax_for(nKT, temporal_blocks(q_frames), kv->Y / 8, kv->X / 8, p);
 }
 
+// Largest number of causal candidates of any query block: the cache's longest
+// stream, all of its temporal blocks.
+static int64_t select_c_stride(const lcsa_kv_cache* kv) {
+  int nKT = 0;
+  for (int b = 0; b < kv->B; ++b) {
+    const int n = static_cast<int>((kv->end[b] >> 1) - (kv->begin[b] >> 1));
+    nKT = n > nKT ? n : nKT;
+  }
+  return static_cast<int64_t>(nKT) * (kv->Y / 8) * (kv->X / 8);
+}
+
+size_t lcsa_select_workspace_bytes(const lcsa_kv_cache* kv, int32_t q_frames) {
+  if (kv == nullptr || q_frames < 1 || kv->B < 1 || kv->B > LCSA_MAX_STREAMS || kv->Y < 8 || kv->X < 8)
+    return 0;
+  const int64_t rows = static_cast<int64_t>(kv->B) * kv->H * temporal_blocks(q_frames) * (kv->Y / 8) * (kv->X / 8);
+  return static_cast<size_t>(rows * select_c_stride(kv)) * sizeof(uint64_t);
+}
+
 lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames, const lcsa_kv_cache* kv,
                                const lcsa_select_params* sp, int32_t* blk_idx, int32_t* blk_cnt,
-                               lcsa_stream_t stream) {
+                               void* workspace, size_t workspace_bytes, lcsa_stream_t stream) {
   lcsa_status s = check_cache(kv);
   if (s != LCSA_OK) return s;
-  if (q_pool == nullptr || sp == nullptr || blk_idx == nullptr || blk_cnt == nullptr)
+  if (q_pool == nullptr || sp == nullptr || blk_idx == nullptr || blk_cnt == nullptr || workspace == nullptr)
     return LCSA_ERR_INVALID_ARG;
-  if (!aligned16(q_pool)) return LCSA_ERR_ALIGN;
+  if (!aligned16(q_pool) || !aligned16(workspace)) return LCSA_ERR_ALIGN;
   if (sp->top_k < 0 || sp->kmax < 1 || !(sp->tie_eps >= 0.0)) return LCSA_ERR_INVALID_ARG;
   if (sp->top_k == 0 && !(sp->density > 0.0 && sp->density <= 1.0)) return LCSA_ERR_INVALID_ARG;
   if (sp->window < 0 || (sp->window > 0 && sp->window % 2 == 0)) return LCSA_ERR_INVALID_ARG;
@@ -319,30 +352,42 @@ lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames, const lcs
     nKT_max = n > nKT_max ? n : nKT_max;
   }
   if (kmax_for(nKT_max, nQT, Hb, Wb, sp) > sp->kmax) return LCSA_ERR_CAPACITY;
-  const int ncand_max = nKT_max * HbWb;
-  const int c_stride = ncand_max + 1;
-  const size_t smem = select_smem_bytes(kv->D, c_stride);
-  if (smem > 227 * 1024) return LCSA_ERR_SHAPE;
+  if (workspace_bytes < lcsa_select_workspace_bytes(kv, q_frames)) return LCSA_ERR_WORKSPACE;
+  const int64_t c_stride = select_c_stride(kv);
+  const int64_t rows = static_cast<int64_t>(kv->B) * kv->H * nQT * HbWb;
+  if (c_stride > 2048 || (c_stride + SC_CANDS - 1) / SC_CANDS > 0x7fffffff ||
+      static_cast<int64_t>(kv->B) * kv->H * nQT > 65535 || rows > 0x7fffffff)
+    return LCSA_ERR_SHAPE;
   int dev;
   unsigned int* err;
   if ((s = device_setup(&dev, &err)) != LCSA_OK) return s;
   SelectParams p{};
   p.q_pool = q_pool;
   p.k_pool = kv->k_pool;
+  p.keys = static_cast<uint64_t*>(workspace);
   p.blk_idx = blk_idx;
   p.blk_cnt = blk_cnt;
-  p.H = kv->H; p.Hb = Hb; p.Wb = Wb; p.nQT = nQT;
+  p.B = kv->B; p.H = kv->H; p.Hb = Hb; p.Wb = Wb; p.nQT = nQT;
   p.cap_blk = kv->cap_frames / 2;
   p.top_k = sp->top_k; p.window = sp->window; p.window_mode = sp->window_mode; p.kmax = sp->kmax;
-  p.c_stride = c_stride;
+  p.c_stride = static_cast<int32_t>(c_stride);
   p.density = sp->density;
   p.tie_eps = sp->tie_eps;
   p.sqrt_d = std::sqrt(static_cast<double>(kv->D));
   p.err = err;
   for (int b = 0; b < kv->B; ++b) { p.kv_begin[b] = kv->begin[b]; p.kv_end[b] = kv->end[b]; }
-  const dim3 grid((HbWb + SEL_ROWS - 1) / SEL_ROWS, nQT, kv->B * kv->H);
-  if (kv->D == 128) select_kernel<128><<<grid, SEL_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
-  else select_kernel<64><<<grid, SEL_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const dim3 sgrid(static_cast<unsigned>((c_stride + SC_CANDS - 1) / SC_CANDS),
+                   static_cast<unsigned>((HbWb + SC_ROWS - 1) / SC_ROWS),
+                   static_cast<unsigned>(kv->B * kv->H * nQT));
+  if (kv->D == 128) score_kernel<128><<<sgrid, SC_THREADS, score_smem_bytes(128), cs>>>(p);
+  else score_kernel<64><<<sgrid, SC_THREADS, score_smem_bytes(64), cs>>>(p);
+  if ((s = launched()) != LCSA_OK) return s;
+  // one CTA per query block, one key per thread up to 1024 candidates, two beyond
+  const int slots = c_stride <= 1024 ? 1 : 2;
+  const unsigned tthreads = static_cast<unsigned>(((c_stride + slots - 1) / slots + 31) / 32 * 32);
+  if (slots == 1) topk_kernel<1><<<static_cast<unsigned>(rows), tthreads, 0, cs>>>(p);
+  else topk_kernel<2><<<static_cast<unsigned>(rows), tthreads, 0, cs>>>(p);
   return launched();
 }
 
@@ -423,6 +468,19 @@ lcsa_status lcsa_debug_stalled_wait(uint64_t limit_ns, lcsa_stream_t stream) {
   if (s != LCSA_OK) return s;
   if (limit_ns == 0 || limit_ns > 10000000000ull) return LCSA_ERR_INVALID_ARG;
   stalled_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, err);
+  return launched();
+}
+
+lcsa_status lcsa_debug_exp2_poly(const float* x, float* y, int64_t n, lcsa_stream_t stream) {
+  if (x == nullptr || y == nullptr || n < 1) return LCSA_ERR_INVALID_ARG;
+  int dev;
+  unsigned int* err;
+  lcsa_status s = device_setup(&dev, &err);
+  if (s != LCSA_OK) return s;
+  const int64_t threads = (n + 1) / 2;
+  const int64_t grid = (threads + 255) / 256;
+  if (grid > 0x7fffffff) return LCSA_ERR_SHAPE;
+  exp2_poly_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   return launched();
 }
 

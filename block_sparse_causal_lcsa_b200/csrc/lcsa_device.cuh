@@ -193,6 +193,13 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
       LCSA_W8(0), LCSA_W8(8), LCSA_W8(16), LCSA_W8(24)
       : "memory");
 }
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      LCSA_W8(0), LCSA_W8(8)
+      : "memory");
+}
 #undef LCSA_R8
 #undef LCSA_W8
 
@@ -209,6 +216,77 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Named barrier over `count` threads (ids 1..15; 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// max of three floats in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Two fp32 lanes in one 64-bit register: packed fma / add (sm_100).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+  return v;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for two lanes on the FMA pipe (x <= 8; x is clamped at -126, so far
+// below that the result is about 2^-126, never a NaN):
+// x = n + f with n = round(x) taken from the low mantissa bits of x + 1.5*2^23
+// and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted for minimax
+// relative error (7.5e-5) with the Remez exchange (fit_exp2_poly.py); 2^n
+// applied by adding n to the exponent field.
+__device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  // with n >= -126 and p(f) in [0.70, 1.42] the exponent field stays >= 0
+  x = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+  const uint64_t neg_magic = f2_pack(-12582912.f, -12582912.f);
+  const uint64_t t = f2_add(x, magic);
+  const uint64_t nf = f2_add(t, neg_magic);                       // round(x), exact
+  const uint64_t f = f2_fma(nf, f2_pack(-1.f, -1.f), x);          // x - round(x), exact
+  uint64_t p = f2_fma(f2_pack(5.517166853e-02f, 5.517166853e-02f), f, f2_pack(2.426111251e-01f, 2.426111251e-01f));
+  p = f2_fma(p, f, f2_pack(6.932609677e-01f, 6.932609677e-01f));
+  p = f2_fma(p, f, f2_pack(9.999280572e-01f, 9.999280572e-01f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  const float r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  const float r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+  return f2_pack(r0, r1);
+}
+
+// Two non-negative floats -> bf16x2 with integer ops (ALU pipe, keeping the
+// special-function pipe free for exponentials): adding 0x8000 to the bit
+// pattern rounds the magnitude to the nearest bf16 (ties upward), then prmt
+// keeps the two high halves (lo in bits 0-15).
+__device__ __forceinline__ uint32_t pack_bf16x2_pos(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo) + 0x8000u;
+  const uint32_t b = __float_as_uint(hi) + 0x8000u;
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -3,45 +3,50 @@
 // keep the top-K block pairs, causal masking; section 2.3: a spatial window
 // per query with a boundary-truncate or boundary-preserve rule).
 //
-// One CTA (4 warps) owns SEL_ROWS query blocks of one (stream, head, temporal
-// block) and all of their causal candidates.
-// Phase 1: each thread takes candidates in turn, streams the candidate's
-//   pooled key row from L2 and scores it against all SEL_ROWS query rows held
-//   in shared memory: SEL_ROWS independent float64 chains, each summed in
-//   channel order with every product rounded before it is added (no fused
-//   multiply-add), then divided by sqrt(D) - the same float64 value as the
-//   definition, bit for bit. Scores become order-preserving 64-bit keys;
-//   blocks outside the window get key 0, below every finite score.
-// Phase 2: one warp per query block finds the K-th largest key exactly with an
-//   8-pass, 8-bit radix select (256-bin shared-memory histogram per pass,
-//   warp suffix scan), then one ascending pass keeps every block above
-//   tau+eps and the lowest-index blocks of the band [tau-eps, tau+eps].
+// Two kernels, joined by a caller-provided workspace of 64-bit keys
+// [rows][c_stride]:
+// score_kernel  one CTA per (8 query blocks) x (64 candidate key blocks) of a
+//   (stream, head, temporal block). The 8 pooled query rows and the 64 pooled
+//   key rows are staged in shared memory (key rows padded to D+1 doubles so
+//   the 32 lanes of a warp, each reading its own row, hit distinct banks);
+//   each thread scores one candidate against 4 rows - 4 independent float64
+//   chains, each summed in channel order with every product rounded before it
+//   is added (no fused multiply-add), then divided by sqrt(D): the same
+//   float64 value as the definition, bit for bit. Scores are stored as
+//   order-preserving 64-bit keys; candidates outside the row's window get
+//   key 0, below every finite score.
+// topk_kernel   one CTA per query block, one or two keys per thread held in
+//   registers (at most 2048 causal candidates): the exact K-th largest key by
+//   a 1-bit radix select (one CTA-wide count per bit from the top, stopping
+//   once a single key matches), then one ascending pass keeps every block
+//   above tau+eps and the lowest-index blocks of the band [tau-eps, tau+eps].
 #pragma once
 
 #include "lcsa_device.cuh"
 
 namespace lcsa {
 
-constexpr int SEL_ROWS = 4;       // query blocks per CTA (one warp each in phase 2)
-constexpr int SEL_THREADS = SEL_ROWS * 32;
+constexpr int SC_ROWS = 8;        // query blocks per score CTA
+constexpr int SC_CANDS = 64;      // candidate key blocks per score CTA
+constexpr int SC_THREADS = 128;   // 64 candidates x 2 groups of 4 rows
 
 struct SelectParams {
   const double* q_pool;   // [B][H][nQT][Hb][Wb][D]
   const double* k_pool;   // ring [B][H][cap_blk][Hb][Wb][D]
+  uint64_t* keys;         // workspace [B*H*nQB][c_stride]
   int32_t* blk_idx;       // [B][H][nQT*Hb*Wb][kmax]
   int32_t* blk_cnt;       // [B][H][nQT*Hb*Wb]
-  int32_t H, Hb, Wb, nQT, cap_blk;
+  int32_t B, H, Hb, Wb, nQT, cap_blk;
   int32_t top_k, window, window_mode, kmax;
-  int32_t c_stride;       // row stride (keys) of the key buffer in shared memory
+  int32_t c_stride;       // row stride (keys) of the workspace = most causal candidates of any row
   double density, tie_eps, sqrt_d;
   unsigned int* err;
   int64_t kv_begin[64];
   int64_t kv_end[64];
 };
 
-__host__ __device__ constexpr size_t select_smem_bytes(int D, int c_stride) {
-  return sizeof(double) * SEL_ROWS * D + sizeof(uint32_t) * SEL_ROWS * 256 +
-         sizeof(uint64_t) * static_cast<size_t>(SEL_ROWS) * c_stride;
+__host__ __device__ constexpr size_t score_smem_bytes(int D) {
+  return sizeof(double) * (static_cast<size_t>(SC_ROWS) * D + static_cast<size_t>(SC_CANDS) * (D + 1));
 }
 
 __device__ __forceinline__ uint64_t order_key(double s) {
@@ -65,96 +70,169 @@ __device__ __forceinline__ void window_bounds(int i, int n, int w, int mode, int
   }
 }
 
+// Candidate range of a stream: the key timeline's oldest cached block and the
+// query time step tq's position in it.
+struct StreamGeom {
+  int64_t m_first;  // absolute index of the oldest cached block
+  int slot0;        // its ring slot
+  int tq_kv;        // key temporal block of query temporal block tq
+  int ncand;        // causal candidates (tq_kv + 1) * Hb * Wb
+};
+
+__device__ __forceinline__ StreamGeom stream_geom(const SelectParams& p, int b, int tq) {
+  StreamGeom g;
+  const int64_t begin = p.kv_begin[b], end = p.kv_end[b];
+  g.m_first = begin >> 1;
+  g.slot0 = static_cast<int>(g.m_first % p.cap_blk);
+  const int nKT = static_cast<int>((end >> 1) - g.m_first);
+  g.tq_kv = nKT - p.nQT + tq;
+  g.ncand = (g.tq_kv + 1) * p.Hb * p.Wb;
+  return g;
+}
+
 template <int D>
-__global__ void __launch_bounds__(SEL_THREADS)
-select_kernel(const __grid_constant__ SelectParams p) {
-  extern __shared__ __align__(16) uint8_t sel_smem[];
-  double* qs = reinterpret_cast<double*>(sel_smem);                       // [R][D]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(qs + SEL_ROWS * D);        // [R][256]
-  uint64_t* keys = reinterpret_cast<uint64_t*>(hist + SEL_ROWS * 256);    // [R][c_stride]
+__global__ void __launch_bounds__(SC_THREADS)
+score_kernel(const __grid_constant__ SelectParams p) {
+  extern __shared__ __align__(16) double sc_smem[];
+  double* qs = sc_smem;                         // [SC_ROWS][D]
+  double* ks = qs + SC_ROWS * D;                // [SC_CANDS][D+1]
 
   const int HbWb = p.Hb * p.Wb;
-  const int bh = blockIdx.z;
-  const int b = bh / p.H;
-  const int tq = blockIdx.y;
-  const int sp0 = blockIdx.x * SEL_ROWS;
-  const int nrows = min(SEL_ROWS, HbWb - sp0);
-  const int64_t begin = p.kv_begin[b], end = p.kv_end[b];
-  const int64_t m_first = begin >> 1;               // oldest cached block (absolute)
-  const int slot0 = static_cast<int>(m_first % p.cap_blk);
-  const int nKT = static_cast<int>((end >> 1) - m_first);
-  const int tq_kv = nKT - p.nQT + tq;               // query time step in the key timeline
-  const int ncand = (tq_kv + 1) * HbWb;             // causal candidates
   const int nQB = p.nQT * HbWb;
+  const int bh = blockIdx.z / p.nQT;
+  const int tq = blockIdx.z % p.nQT;
+  const int b = bh / p.H;
+  const int sp0 = blockIdx.y * SC_ROWS;
+  const int nrows = min(SC_ROWS, HbWb - sp0);
+  const StreamGeom g = stream_geom(p, b, tq);
+  const int c0 = blockIdx.x * SC_CANDS;
+  if (c0 >= g.ncand || nrows <= 0) return;
+  const int ncur = min(SC_CANDS, g.ncand - c0);
   const int tid = threadIdx.x;
 
-  // Pull every candidate's pooled key row toward L2 up front, so the scoring
-  // loop below waits on L2 rather than on DRAM (rows are D*8 bytes).
-  {
-    constexpr int LINES = D * 8 / 128;
-    for (int e = tid; e < ncand * LINES; e += SEL_THREADS) {
-      const int j = e / LINES, l = e % LINES;
+  const int warp = tid >> 5, lane = tid & 31;
+  constexpr int V2 = D / 2;                       // 16-byte vectors per pooled row
+  constexpr int PER_LANE = V2 / 32;               // vectors per lane per row
+  constexpr int ROWS_PER_WARP = SC_CANDS / (SC_THREADS / 32);
+  // query rows: warp w stages rows w, w+4 (plain copy, zero beyond nrows)
+  const double2* qsrc = reinterpret_cast<const double2*>(
+      p.q_pool + (static_cast<int64_t>(bh) * nQB + tq * HbWb + sp0) * D);
+#pragma unroll
+  for (int rr = warp; rr < SC_ROWS; rr += SC_THREADS / 32) {
+#pragma unroll
+    for (int v = 0; v < PER_LANE; ++v) {
+      const int e = v * 32 + lane;
+      const double2 x = rr < nrows ? __ldg(qsrc + rr * V2 + e) : make_double2(0.0, 0.0);
+      qs[rr * D + 2 * e] = x.x;
+      qs[rr * D + 2 * e + 1] = x.y;
+    }
+  }
+  // candidate rows: warp w stages rows w*16 .. w*16+15, all loads issued before
+  // any store so that the L2 round trips overlap
+  double2 buf[ROWS_PER_WARP][PER_LANE];
+#pragma unroll
+  for (int i = 0; i < ROWS_PER_WARP; ++i) {
+    const int cc = warp * ROWS_PER_WARP + i;
+    const int j = c0 + cc;
+    if (cc < ncur) {
       const int tk = j / HbWb, spk = j - tk * HbWb;
-      const int slot = (slot0 + tk) % p.cap_blk;
-      const double* line = p.k_pool + ((static_cast<int64_t>(bh) * p.cap_blk + slot) * HbWb + spk) * D + l * 16;
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(line));
+      const int slot = (g.slot0 + tk) % p.cap_blk;
+      const double2* src = reinterpret_cast<const double2*>(
+          p.k_pool + ((static_cast<int64_t>(bh) * p.cap_blk + slot) * HbWb + spk) * D);
+#pragma unroll
+      for (int v = 0; v < PER_LANE; ++v) buf[i][v] = __ldg(src + v * 32 + lane);
+    } else {
+#pragma unroll
+      for (int v = 0; v < PER_LANE; ++v) buf[i][v] = make_double2(0.0, 0.0);
     }
   }
-
-  const double* qsrc = p.q_pool + (static_cast<int64_t>(bh) * nQB + tq * HbWb + sp0) * D;
-  for (int e = tid; e < SEL_ROWS * D; e += SEL_THREADS)
-    qs[e] = e < nrows * D ? qsrc[e] : 0.0;
-
-  int y0[SEL_ROWS], y1[SEL_ROWS], x0[SEL_ROWS], x1[SEL_ROWS];
 #pragma unroll
-  for (int r = 0; r < SEL_ROWS; ++r) {
-    const int sp = min(sp0 + r, HbWb - 1);
-    window_bounds(sp / p.Wb, p.Hb, p.window, p.window_mode, y0[r], y1[r]);
-    window_bounds(sp % p.Wb, p.Wb, p.window, p.window_mode, x0[r], x1[r]);
-  }
-  __syncthreads();
-
-  // Phase 1: keys of all causal candidates for the CTA's rows.
-  const double2* q2 = reinterpret_cast<const double2*>(qs);
-  for (int j = tid; j < ncand; j += SEL_THREADS) {
-    const int tk = j / HbWb, spk = j - tk * HbWb;
-    const int yk = spk / p.Wb, xk = spk - yk * p.Wb;
-    const int slot = (slot0 + tk) % p.cap_blk;
-    const double2* kr = reinterpret_cast<const double2*>(
-        p.k_pool + ((static_cast<int64_t>(bh) * p.cap_blk + slot) * HbWb + spk) * D);
-    double s[SEL_ROWS];
+  for (int i = 0; i < ROWS_PER_WARP; ++i) {
+    const int cc = warp * ROWS_PER_WARP + i;
 #pragma unroll
-    for (int r = 0; r < SEL_ROWS; ++r) s[r] = 0.0;
-#pragma unroll 16
-    for (int c2 = 0; c2 < D / 2; ++c2) {
-      const double2 kv = __ldg(kr + c2);
-#pragma unroll
-      for (int r = 0; r < SEL_ROWS; ++r) {
-        const double2 qv = q2[r * (D / 2) + c2];
-        s[r] = __dadd_rn(s[r], __dmul_rn(qv.x, kv.x));
-        s[r] = __dadd_rn(s[r], __dmul_rn(qv.y, kv.y));
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < SEL_ROWS; ++r) {
-      if (r < nrows) {
-        const bool ok = yk >= y0[r] && yk < y1[r] && xk >= x0[r] && xk < x1[r];
-        // adding +0.0 turns -0.0 into +0.0, so equal scores get equal keys
-        const double sc = __dadd_rn(__ddiv_rn(s[r], p.sqrt_d), 0.0);
-        keys[r * p.c_stride + j] = ok ? order_key(sc) : 0ull;
-      }
+    for (int v = 0; v < PER_LANE; ++v) {
+      const int e = v * 32 + lane;
+      ks[cc * (D + 1) + 2 * e] = buf[i][v].x;
+      ks[cc * (D + 1) + 2 * e + 1] = buf[i][v].y;
     }
   }
   __syncthreads();
 
-  // Phase 2: one warp per query block.
-  const int r = tid >> 5;
-  if (r >= nrows) return;
-  const int lane = tid & 31;
-  int wy0, wy1, wx0, wx1;
-  window_bounds((sp0 + r) / p.Wb, p.Hb, p.window, p.window_mode, wy0, wy1);
-  window_bounds((sp0 + r) % p.Wb, p.Wb, p.window, p.window_mode, wx0, wx1);
-  const int C = (tq_kv + 1) * (wy1 - wy0) * (wx1 - wx0);
+  const int cc = tid % SC_CANDS;
+  const int r0 = (tid / SC_CANDS) * 4;
+  if (cc >= ncur) return;
+  const double* kr = ks + cc * (D + 1);
+  double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+#pragma unroll 8
+  for (int c = 0; c < D; ++c) {
+    const double kv = kr[c];
+    s0 = __dadd_rn(s0, __dmul_rn(qs[(r0 + 0) * D + c], kv));
+    s1 = __dadd_rn(s1, __dmul_rn(qs[(r0 + 1) * D + c], kv));
+    s2 = __dadd_rn(s2, __dmul_rn(qs[(r0 + 2) * D + c], kv));
+    s3 = __dadd_rn(s3, __dmul_rn(qs[(r0 + 3) * D + c], kv));
+  }
+  const int j = c0 + cc;
+  const int spk = j % HbWb;
+  const int yk = spk / p.Wb, xk = spk - yk * p.Wb;
+  const double sv[4] = {s0, s1, s2, s3};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + i;
+    if (r >= nrows) break;
+    const int sp = sp0 + r;
+    int y0, y1, x0, x1;
+    window_bounds(sp / p.Wb, p.Hb, p.window, p.window_mode, y0, y1);
+    window_bounds(sp % p.Wb, p.Wb, p.window, p.window_mode, x0, x1);
+    const bool ok = yk >= y0 && yk < y1 && xk >= x0 && xk < x1;
+    // adding +0.0 turns -0.0 into +0.0, so equal scores get equal keys
+    const double sc = __dadd_rn(__ddiv_rn(sv[i], p.sqrt_d), 0.0);
+    const int64_t row = static_cast<int64_t>(bh) * nQB + tq * HbWb + sp;
+    p.keys[row * p.c_stride + j] = ok ? order_key(sc) : 0ull;
+  }
+}
+
+// Exclusive prefix count of f over the CTA in thread order, and its total.
+__device__ __forceinline__ int cta_excl_count(bool f, int& total, int* wsum) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  const uint32_t m = __ballot_sync(0xffffffffu, f);
+  if (lane == 0) wsum[warp] = __popc(m);
+  __syncthreads();
+  int before = 0, tot = 0;
+  for (int w = 0; w < nwarps; ++w) {
+    const int v = wsum[w];
+    before += w < warp ? v : 0;
+    tot += v;
+  }
+  __syncthreads();  // wsum is reused by the next call
+  total = tot;
+  return before + __popc(m & ((1u << lane) - 1u));
+}
+
+// One CTA per query block; candidate j = s*blockDim.x + threadIdx.x sits in
+// slot s of that thread (a row has at most SLOTS*blockDim.x candidates).
+template <int SLOTS>
+__global__ void __launch_bounds__(1024)
+topk_kernel(const __grid_constant__ SelectParams p) {
+  __shared__ int wsum[32];
+  __shared__ uint64_t last_key;
+  const int HbWb = p.Hb * p.Wb;
+  const int nQB = p.nQT * HbWb;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int64_t row = blockIdx.x;
+  const int bh = static_cast<int>(row / nQB);
+  const int qi = static_cast<int>(row % nQB);
+  const int tq = qi / HbWb, sp = qi % HbWb;
+  const StreamGeom g = stream_geom(p, bh / p.H, tq);
+  const int ncand = g.ncand;
+  if (ncand > SLOTS * nt) {  // the launch is sized for the longest stream
+    if (tid == 0) atomicOr(p.err, DEVERR_BOUNDS);
+    return;
+  }
+  int y0, y1, x0, x1;
+  window_bounds(sp / p.Wb, p.Hb, p.window, p.window_mode, y0, y1);
+  window_bounds(sp % p.Wb, p.Wb, p.window, p.window_mode, x0, x1);
+  const int C = (g.tq_kv + 1) * (y1 - y0) * (x1 - x0);
   int K;
   if (p.top_k > 0) {
     K = min(C, p.top_k);
@@ -162,86 +240,77 @@ select_kernel(const __grid_constant__ SelectParams p) {
     const double kd = ceil(__dmul_rn(p.density, static_cast<double>(C)));
     K = min(C, max(1, static_cast<int>(kd)));
   }
-  const uint64_t* krow = keys + r * p.c_stride;
-  uint32_t* h = hist + r * 256;
+  const uint64_t* krow = p.keys + row * p.c_stride;
+  if (tid == 0) last_key = 0ull;  // ordered by the counting barriers below
+  uint64_t key[SLOTS];
+  bool act[SLOTS];
+  int nact = 0;
+#pragma unroll
+  for (int s = 0; s < SLOTS; ++s) {
+    const int j = s * nt + tid;
+    key[s] = j < ncand ? krow[j] : 0ull;
+    act[s] = key[s] != 0ull;  // window-masked candidates are not ranked
+    nact += __syncthreads_count(act[s]);
+  }
 
-  // Exact K-th largest key, 8 bits at a time from the top.
-  uint64_t prefix = 0, pmask = 0;
+  // Exact K-th largest key, one bit at a time from the top: the CTA counts
+  // the still-matching keys that have the bit set; the K-th largest has it
+  // iff at least krem of them do. Stops early once one key remains.
+  uint64_t prefix = 0;
   int krem = K;
-  for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int i = lane; i < 256; i += 32) h[i] = 0u;
-    __syncwarp();
-    for (int j = lane; j < ncand; j += 32) {
-      const uint64_t key = krow[j];
-      if (key != 0ull && (key & pmask) == prefix)
-        atomicAdd(&h[static_cast<int>((key >> shift) & 255u)], 1u);
-    }
-    __syncwarp();
-    uint32_t c[8];
-    int local = 0;
+  int bit = 63;
+  for (; bit >= 0 && nact > 1; --bit) {
+    int cnt = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      c[i] = h[8 * lane + i];
-      local += static_cast<int>(c[i]);
+    for (int s = 0; s < SLOTS; ++s) cnt += __syncthreads_count(act[s] && ((key[s] >> bit) & 1ull));
+    const uint64_t chosen = cnt >= krem ? 1ull : 0ull;
+    if (chosen) {
+      nact = cnt;
+    } else {
+      krem -= cnt;
+      nact -= cnt;
     }
-    int suf = local;  // keys of this prefix whose digit falls in bins >= 8*lane
+    prefix |= chosen << bit;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_down_sync(0xffffffffu, suf, o);
-      if (lane + o < 32) suf += v;
-    }
-    const int above_lane = suf - local;
-    const uint32_t hit = __ballot_sync(0xffffffffu, above_lane < krem && suf >= krem);
-    const int src = __ffs(hit) - 1;
-    int digit = 0, knew = 0;
-    if (lane == src) {
-      int acc = above_lane;
+    for (int s = 0; s < SLOTS; ++s) act[s] = act[s] && ((key[s] >> bit) & 1ull) == chosen;
+  }
+  if (bit >= 0) {  // a single key matches the prefix: it is the K-th largest
 #pragma unroll
-      for (int i = 7; i >= 0; --i) {
-        if (acc + static_cast<int>(c[i]) >= krem) {
-          digit = 8 * lane + i;
-          knew = krem - acc;
-          break;
-        }
-        acc += static_cast<int>(c[i]);
-      }
-    }
-    digit = __shfl_sync(0xffffffffu, digit, src);
-    krem = __shfl_sync(0xffffffffu, knew, src);
-    prefix |= static_cast<uint64_t>(digit) << shift;
-    pmask |= static_cast<uint64_t>(255) << shift;
-    __syncwarp();
+    for (int s = 0; s < SLOTS; ++s)
+      if (act[s]) last_key = key[s];
+    __syncthreads();
+    prefix = last_key;
   }
   const double tau = key_value(prefix);
   const uint64_t k_hi = order_key(__dadd_rn(tau, p.tie_eps));
   const uint64_t k_lo = order_key(__dsub_rn(tau, p.tie_eps));
   int above = 0;
-  for (int j = lane; j < ncand; j += 32) above += krow[j] > k_hi ? 1 : 0;
-  above = __reduce_add_sync(0xffffffffu, above);
+#pragma unroll
+  for (int s = 0; s < SLOTS; ++s) above += __syncthreads_count(key[s] > k_hi);
   const int need = K - above;
 
-  const int64_t row = static_cast<int64_t>(bh) * nQB + tq * HbWb + sp0 + r;
+  // Keep everything above the band and the lowest-index band members; write
+  // the kept ids in ascending order.
   int32_t* out = p.blk_idx + row * p.kmax;
-  const uint32_t lt_mask = (1u << lane) - 1u;
   int n_band = 0, n_sel = 0;
-  for (int j0 = 0; j0 < ncand; j0 += 32) {
-    const int j = j0 + lane;
-    const uint64_t key = j < ncand ? krow[j] : 0ull;
-    const bool in_above = key > k_hi;
-    const bool in_band = key >= k_lo && key <= k_hi;
-    const uint32_t band_mask = __ballot_sync(0xffffffffu, in_band);
-    const bool take = in_above || (in_band && (n_band + __popc(band_mask & lt_mask)) < need);
-    const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
+#pragma unroll
+  for (int s = 0; s < SLOTS; ++s) {
+    const int j = s * nt + tid;
+    const bool in_above = key[s] > k_hi;
+    const bool in_band = key[s] >= k_lo && key[s] <= k_hi;
+    int band_tot, sel_tot;
+    const int band_before = cta_excl_count(in_band, band_tot, wsum);
+    const bool take = in_above || (in_band && n_band + band_before < need);
+    const int pos = n_sel + cta_excl_count(take, sel_tot, wsum);
     if (take) {
-      const int pos = n_sel + __popc(take_mask & lt_mask);
       if (pos < p.kmax) out[pos] = j;
       else atomicOr(p.err, DEVERR_BOUNDS);
     }
-    n_band += __popc(band_mask);
-    n_sel += __popc(take_mask);
+    n_band += band_tot;
+    n_sel += sel_tot;
   }
-  for (int pos = K + lane; pos < p.kmax; pos += 32) out[pos] = -1;
-  if (lane == 0) p.blk_cnt[row] = K;
+  for (int pos = K + tid; pos < p.kmax; pos += nt) out[pos] = -1;
+  if (tid == 0) p.blk_cnt[row] = K;
 }
 
 }  // namespace lcsa

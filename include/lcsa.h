@@ -65,7 +65,7 @@ typedef enum lcsa_status {
   LCSA_ERR_SHAPE = -2,        /* extents inconsistent or unsupported           */
   LCSA_ERR_ALIGN = -3,        /* pointer or stride misaligned                  */
   LCSA_ERR_CAPACITY = -4,     /* KV cache or blk_idx row capacity exceeded     */
-  LCSA_ERR_WORKSPACE = -5,    /* reserved                                      */
+  LCSA_ERR_WORKSPACE = -5,    /* workspace missing or too small                */
   LCSA_ERR_CUDA = -6,         /* a CUDA runtime/driver call failed             */
   LCSA_ERR_TIMEOUT = -7,      /* a kernel wait gave up (device error word)     */
   LCSA_ERR_DEVICE_BOUNDS = -8 /* a kernel saw an out-of-range block id         */
@@ -182,6 +182,14 @@ LCSA_API int32_t lcsa_select_kmax(const lcsa_kv_cache* kv, int32_t q_frames,
                          const lcsa_select_params* p);
 
 /*
+ * Bytes of device workspace lcsa_select_blocks needs for this cache state and
+ * q_frames query frames: one 64-bit key per (query block, causal candidate),
+ * B*H*ceil(q_frames/2)*Hb*Wb rows of (longest stream's temporal blocks)*Hb*Wb.
+ * Returns 0 on invalid arguments.
+ */
+LCSA_API size_t lcsa_select_workspace_bytes(const lcsa_kv_cache* kv, int32_t q_frames);
+
+/*
  * lcsa_select_blocks - coarse block map, masks and top-K (section 2.2,
  * stage 2: "coarse block-to-block attention map ... keep only the most
  * relevant top-K block pairs", causal masking; section 2.3 locality window).
@@ -194,16 +202,22 @@ LCSA_API int32_t lcsa_select_kmax(const lcsa_kv_cache* kv, int32_t q_frames,
  *           counted from the stream's oldest cached block), unused tail
  *           entries are -1.
  * blk_cnt   device, int32 [B][H][nQB]; K_i per row.
+ * workspace device scratch of at least lcsa_select_workspace_bytes() bytes,
+ *           16-byte aligned, owned by the caller; its contents are undefined
+ *           afterwards and two calls in flight must not share it.
  * Scores are s_ij = (qbar_i . kbar_j) / sqrt(D) in float64, the dot product
  * summed in channel order with every product rounded before it is added, so
  * selections are reproducible bit for bit. Key block j is a candidate of
  * query block i iff t_j <= t_i (block-level causality) and j lies in i's
- * window.
+ * window. At most 2048 causal candidates per query block (longest stream's
+ * temporal blocks x Hb x Wb), else LCSA_ERR_SHAPE. LCSA_ERR_WORKSPACE if
+ * workspace_bytes is too small.
  */
 LCSA_API lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames,
                                const lcsa_kv_cache* kv,
                                const lcsa_select_params* p, int32_t* blk_idx,
-                               int32_t* blk_cnt, lcsa_stream_t stream);
+                               int32_t* blk_cnt, void* workspace,
+                               size_t workspace_bytes, lcsa_stream_t stream);
 
 /*
  * lcsa_sparse_attn_fwd - attention inside the kept blocks (section 2.2,
@@ -248,6 +262,15 @@ LCSA_API lcsa_status lcsa_debug_set_wait_limit_ns(uint64_t ns);
  * the context stays usable. No fault, trap or hang is involved.
  */
 LCSA_API lcsa_status lcsa_debug_stalled_wait(uint64_t limit_ns, lcsa_stream_t stream);
+
+/*
+ * Test hook: y[i] = 2^x[i] (x[i] <= 8) evaluated with the polynomial the
+ * attention kernel uses on the FMA pipe for a quarter of its exponentials
+ * (range reduction x = n + f, |f| <= 1/2, degree-3 minimax polynomial for
+ * 2^f, exponent add for 2^n). x, y: device float32 arrays of n elements.
+ */
+LCSA_API lcsa_status lcsa_debug_exp2_poly(const float* x, float* y, int64_t n,
+                                          lcsa_stream_t stream);
 
 #ifdef __cplusplus
 }

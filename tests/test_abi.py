@@ -11,12 +11,22 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
+def _build_module():
+    # loaded by path: importing the package would load the (possibly stale) library first
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location(
+        "lcsa_build", os.path.join(ROOT, "block_sparse_causal_lcsa_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
 @pytest.fixture(scope="module")
 def lib():
-    from block_sparse_causal_lcsa_b200 import build as b
+    _build_module().build()
     from block_sparse_causal_lcsa_b200 import _abi
 
-    b.build()
     return _abi.load()
 
 
@@ -71,16 +81,21 @@ def test_argument_errors_before_any_launch(lib):
     kv.k, kv.v, kv.k_pool = 0x1000, 0x2000, 0x3000
     kv.B, kv.H, kv.cap_frames, kv.Y, kv.X, kv.D = 1, 1, 5, 16, 16, 128
     sp = _abi.SelectParamsStruct(2, 0, 0, 2, 0.0, 1e-5)
-    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, None) == _abi.ERR_SHAPE
+    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, 0x7000, 1 << 20, None) == _abi.ERR_SHAPE
     kv.cap_frames = 6
     kv.end[0] = 3  # end must stay even
-    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, None) == _abi.ERR_INVALID_ARG
+    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, 0x7000, 1 << 20, None) == _abi.ERR_INVALID_ARG
     kv.end[0] = 6
     sp.window = 4  # even window
-    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, None) == _abi.ERR_INVALID_ARG
+    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, 0x7000, 1 << 20, None) == _abi.ERR_INVALID_ARG
     sp.window = 0
+    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, 0x7000, 8, None) == _abi.ERR_WORKSPACE
     sp.kmax = 1  # K = 2 does not fit
-    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, None) == _abi.ERR_CAPACITY
+    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, 0x7000, 1 << 20, None) == _abi.ERR_CAPACITY
+    # more than 2048 causal candidates per query block: 513 temporal blocks x 4
+    sp.kmax = 2
+    kv.cap_frames, kv.end[0] = 1026, 1026
+    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, 0x7000, 1 << 40, None) == _abi.ERR_SHAPE
 
 
 def test_select_kmax_host_rule(lib):
@@ -93,3 +108,5 @@ def test_select_kmax_host_rule(lib):
     kv.Y, kv.X = 96, 168
     sp.window = 9
     assert lib.lcsa_select_kmax(C.byref(kv), 2, C.byref(sp)) == 34  # 243 candidates
+    # workspace: 12 heads x 252 query blocks x 756 causal candidates x 8 bytes
+    assert lib.lcsa_select_workspace_bytes(C.byref(kv), 2) == 12 * 252 * 756 * 8

@@ -104,6 +104,18 @@ def test_full_clip_selection_and_sampled_output(lc):
             check_output(O[0, h], ro, L[0, h], rl, "clip h%d" % h)
 
 
+@pytest.mark.parametrize("past", [250, 372])
+def test_long_cache_many_candidates(lc, past):
+    """A long cache: 756 and 1122 causal candidates per query block, so the
+    top-K keeps 32 and 64 keys per lane in registers."""
+    w = li.Workload("long", B=1, H=2, D=128, Y=16, X=24, q_frames=2, kv_past=(past,),
+                    cap_frames=past + 2, density=0.05, seed=71)
+    x = li.make_inputs(w)
+    g = run_gpu(lc, w, x)
+    assert g["err"] == 0
+    compare_all(w, x, g)
+
+
 def test_attention_on_oracle_mask(lc):
     """O computed from the oracle's own block lists (selection errors excluded)."""
     w = li.small_variant(li.workload("chunk"), H=2, Y=24, X=40)
@@ -252,3 +264,31 @@ def test_out_of_range_block_id_is_reported(lc):
     bad[0, 0, 0, 0] = 10_000
     lc.sparse_attn_fwd(g["q"], g["cache"], bad, step.blk_cnt)
     assert lc.last_device_error() == -8
+
+
+def test_exp2_polynomial_error_bound(lc):
+    """The FMA-pipe 2^x used for a quarter of the softmax exponentials stays
+    within its fitted relative error bound (7.5e-5, plus float32 rounding)
+    against torch's float32 exp2, over the softmax's argument range."""
+    x = torch.linspace(-100.0, 8.0, 1_000_001, device="cuda", dtype=torch.float32)
+    y = lc.debug_exp2_poly(x)
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref).abs() / ref).max().item()
+    assert rel < 1.0e-4
+    # far below the range it returns (almost) zero, never garbage
+    z = lc.debug_exp2_poly(torch.tensor([-float("inf"), -1e30, -300.0, -127.0, -126.4], device="cuda"))
+    assert torch.isfinite(z).all() and (z >= 0).all() and (z < 1e-37).all()
+
+
+def test_wide_logit_range(lc):
+    """Q scaled by 30: logits spread over hundreds of log2 units, so the
+    exponentials see arguments far below the polynomial's clamp and the lazy
+    rescale of O triggers; the output still matches the oracle."""
+    w = li.Workload("wide", B=1, H=2, D=128, Y=16, X=24, q_frames=2, kv_past=(4,), cap_frames=6,
+                    density=0.5, seed=61)
+    x = li.make_inputs(w)
+    x["q"] = (x["q"].float() * 30.0).to(torch.bfloat16)
+    g = run_gpu(lc, w, x)
+    assert g["err"] == 0
+    assert np.isfinite(g["O"]).all()
+    compare_all(w, x, g)
