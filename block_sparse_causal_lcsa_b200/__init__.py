@@ -19,6 +19,7 @@ from .api import (  # noqa: F401
     last_device_error,
     pool_qk,
     select_blocks,
+    select_blocks_noalloc,
     select_kmax,
     select_workspace_bytes,
     sparse_attn_fwd,

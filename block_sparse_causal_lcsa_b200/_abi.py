@@ -22,6 +22,8 @@ ERR_WORKSPACE = -5
 ERR_CUDA = -6
 ERR_TIMEOUT = -7
 ERR_DEVICE_BOUNDS = -8
+ERR_SCRATCH_LIMIT = -9
+SELECT_STATIC_SCRATCH_BYTES = 8 << 20
 
 WINDOW_TRUNCATE = 0
 WINDOW_PRESERVE = 1
@@ -68,6 +70,9 @@ PROTOTYPES = {
     "lcsa_select_blocks": (C.c_int, [C.c_void_p, C.c_int32, C.POINTER(KVCacheStruct),
                                      C.POINTER(SelectParamsStruct), C.c_void_p, C.c_void_p,
                                      C.c_void_p, C.c_size_t, C.c_void_p]),
+    "lcsa_select_blocks_noalloc": (C.c_int, [C.c_void_p, C.c_int32, C.POINTER(KVCacheStruct),
+                                             C.POINTER(SelectParamsStruct), C.c_void_p, C.c_void_p,
+                                             C.c_void_p]),
     "lcsa_sparse_attn_fwd": (C.c_int, [C.POINTER(Tensor), C.POINTER(KVCacheStruct), C.c_void_p,
                                        C.c_void_p, C.c_int32, C.POINTER(Tensor), C.c_void_p,
                                        C.c_void_p]),

@@ -190,6 +190,27 @@ def select_blocks(q_pool: torch.Tensor, q_frames: int, cache: KVCache, params: S
     return blk_idx, blk_cnt
 
 
+def select_blocks_noalloc(q_pool: torch.Tensor, q_frames: int, cache: KVCache, params: SelectParams,
+                          blk_idx: torch.Tensor, blk_cnt: torch.Tensor,
+                          stream: Optional[torch.cuda.Stream] = None):
+    """select_blocks into caller-given outputs, with the library's fixed
+    scratch array in place of a workspace: nothing is allocated, so it suits
+    callers that may not allocate device memory while they run. kmax is
+    blk_idx.shape[-1]. Raises LcsaError(ERR_SCRATCH_LIMIT) when the selection
+    needs more than SELECT_STATIC_SCRATCH_BYTES of scratch; calls that overlap
+    on the GPU share that scratch and must be serialised."""
+    if q_pool.dtype != torch.float64 or not q_pool.is_contiguous():
+        raise ValueError("q_pool must be contiguous float64")
+    if not blk_idx.is_contiguous() or not blk_cnt.is_contiguous():
+        raise ValueError("blk_idx and blk_cnt must be contiguous")
+    sp = params.struct(blk_idx.shape[-1])
+    _check(_lib.lcsa_select_blocks_noalloc(q_pool.data_ptr(), q_frames, C.byref(cache.struct),
+                                           C.byref(sp), blk_idx.data_ptr(), blk_cnt.data_ptr(),
+                                           _stream(stream)),
+           "lcsa_select_blocks_noalloc")
+    return blk_idx, blk_cnt
+
+
 def sparse_attn_fwd(q: torch.Tensor, cache: KVCache, blk_idx: torch.Tensor, blk_cnt: torch.Tensor,
                     o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                     with_lse: bool = True, stream: Optional[torch.cuda.Stream] = None):

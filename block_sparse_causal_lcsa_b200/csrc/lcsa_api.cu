@@ -1,7 +1,8 @@
 // Host side of liblcsa.so: the C ABI declared in include/lcsa.h. Validates
 // every argument before launching, encodes the TMA tensor maps, sizes the
 // grids and launches the sm_100a kernels on the caller's stream. Allocates no
-// memory: the only device state of the library is its per-device error word.
+// memory: the device state of the library is its per-device error word and
+// the fixed scratch array of lcsa_select_blocks_noalloc.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -14,6 +15,12 @@
 #include "kv_append.cuh"
 #include "pool.cuh"
 #include "select.cuh"
+
+// Scratch of lcsa_select_blocks_noalloc: the score keys that the caller's
+// workspace holds in lcsa_select_blocks. A module-scope array, so it exists on
+// every device that loads this library's kernels, until the process exits.
+// In host code the name is only a handle for cudaGetSymbolAddress.
+static __device__ __align__(256) uint64_t lcsa_select_scratch[LCSA_SELECT_STATIC_SCRATCH_BYTES / sizeof(uint64_t)];
 
 namespace lcsa {
 
@@ -189,6 +196,7 @@ const char* lcsa_status_string(lcsa_status s) {
     case LCSA_ERR_CUDA: return "CUDA error";
     case LCSA_ERR_TIMEOUT: return "a kernel wait timed out";
     case LCSA_ERR_DEVICE_BOUNDS: return "a kernel saw an out-of-range block id";
+    case LCSA_ERR_SCRATCH_LIMIT: return "request exceeds the library's fixed scratch array";
   }
   return "unknown status";
 }
@@ -389,6 +397,35 @@ lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames, const lcs
   if (slots == 1) topk_kernel<1><<<static_cast<unsigned>(rows), tthreads, 0, cs>>>(p);
   else topk_kernel<2><<<static_cast<unsigned>(rows), tthreads, 0, cs>>>(p);
   return launched();
+}
+
+// Device addresses of lcsa_select_scratch, looked up once per device.
+static std::mutex g_scratch_mu;
+static void* g_scratch_ptr[64] = {};
+
+lcsa_status lcsa_select_blocks_noalloc(const double* q_pool, int32_t q_frames, const lcsa_kv_cache* kv,
+                                       const lcsa_select_params* sp, int32_t* blk_idx, int32_t* blk_cnt,
+                                       lcsa_stream_t stream) {
+  if (q_pool == nullptr || kv == nullptr || sp == nullptr || blk_idx == nullptr || blk_cnt == nullptr)
+    return LCSA_ERR_INVALID_ARG;
+  if (lcsa_select_workspace_bytes(kv, q_frames) > LCSA_SELECT_STATIC_SCRATCH_BYTES)
+    return LCSA_ERR_SCRATCH_LIMIT;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LCSA_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+      void* ptr = nullptr;  // this device is current: the address is its copy's
+      if (cudaGetSymbolAddress(&ptr, lcsa_select_scratch) != cudaSuccess || ptr == nullptr)
+        return LCSA_ERR_CUDA;
+      g_scratch_ptr[dev] = ptr;
+    }
+    scratch = g_scratch_ptr[dev];
+  }
+  // the same validation, kernels and results as the workspace entry point
+  return lcsa_select_blocks(q_pool, q_frames, kv, sp, blk_idx, blk_cnt, scratch,
+                            LCSA_SELECT_STATIC_SCRATCH_BYTES, stream);
 }
 
 lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_cache* kv, const int32_t* blk_idx,

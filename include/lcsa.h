@@ -17,7 +17,9 @@
  * Conventions
  * - Memory: the caller owns every buffer. The library allocates no device or
  *   host memory (the attention kernel allocates tensor memory on the SM for
- *   its own lifetime only). A call writes only its output arguments.
+ *   its own lifetime only). Its only device state is a per-device error word
+ *   and the fixed scratch array of lcsa_select_blocks_noalloc. A call writes
+ *   only its output arguments (and that array).
  * - Pointers named "device" must be CUDA device pointers on the current
  *   device; all others are host pointers.
  * - Errors: argument and shape errors are returned synchronously, before any
@@ -68,7 +70,8 @@ typedef enum lcsa_status {
   LCSA_ERR_WORKSPACE = -5,    /* workspace missing or too small                */
   LCSA_ERR_CUDA = -6,         /* a CUDA runtime/driver call failed             */
   LCSA_ERR_TIMEOUT = -7,      /* a kernel wait gave up (device error word)     */
-  LCSA_ERR_DEVICE_BOUNDS = -8 /* a kernel saw an out-of-range block id         */
+  LCSA_ERR_DEVICE_BOUNDS = -8, /* a kernel saw an out-of-range block id        */
+  LCSA_ERR_SCRATCH_LIMIT = -9  /* request exceeds the library's fixed scratch   */
 } lcsa_status;
 
 enum { LCSA_WINDOW_TRUNCATE = 0, LCSA_WINDOW_PRESERVE = 1 };
@@ -218,6 +221,45 @@ LCSA_API lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames,
                                const lcsa_select_params* p, int32_t* blk_idx,
                                int32_t* blk_cnt, void* workspace,
                                size_t workspace_bytes, lcsa_stream_t stream);
+
+/*
+ * lcsa_select_blocks_noalloc - lcsa_select_blocks with library-owned scratch.
+ *
+ * The paper has no counterpart to this call. It is for callers that cannot
+ * allocate device memory for a workspace: a plugin or engine whose device
+ * memory is all owned by a host framework's pool and that has nothing to
+ * hand out per call, or a real-time frame loop that must never call
+ * cudaMalloc, because an allocation can synchronise the device and stall
+ * the stream. The caller still provides q_pool, kv, blk_idx and blk_cnt,
+ * with the same meaning, layout and results as lcsa_select_blocks.
+ *
+ * Scratch: a fixed device array of LCSA_SELECT_STATIC_SCRATCH_BYTES (8 MiB)
+ * inside the library, used in place of the workspace. It exists on every
+ * GPU where the library's kernels are loaded and stays there until the
+ * process exits. The call allocates nothing: no cudaMalloc, cudaFree or
+ * allocating library routine.
+ * - The first call on a device, with that device current, looks up the
+ *   array's device address (cudaGetSymbolAddress). Make that first call
+ *   before any stream capture begins.
+ * - All calls share the one array and it keeps the previous call's contents.
+ *   Nothing in it has to start at zero: every entry the selection reads was
+ *   written earlier in the same call.
+ * - Calls whose work overlaps on the GPU (different streams, several host
+ *   threads) race on the array. Keep them ordered on one stream or otherwise
+ *   serialised.
+ * Limit: lcsa_select_workspace_bytes(kv, q_frames) must not exceed
+ * LCSA_SELECT_STATIC_SCRATCH_BYTES, else LCSA_ERR_SCRATCH_LIMIT, returned
+ * before any device work. Four streams of 768x1408 frames (12 heads, an
+ * 8-frame cache) need 6.7 MB and fit; one 1536x2816 stream with a 6-frame
+ * cache needs 18.3 MB and does not.
+ * Other errors are those of lcsa_select_blocks (LCSA_ERR_CUDA also if the
+ * address look-up fails).
+ */
+#define LCSA_SELECT_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+LCSA_API lcsa_status lcsa_select_blocks_noalloc(const double* q_pool, int32_t q_frames,
+                                       const lcsa_kv_cache* kv,
+                                       const lcsa_select_params* p, int32_t* blk_idx,
+                                       int32_t* blk_cnt, lcsa_stream_t stream);
 
 /*
  * lcsa_sparse_attn_fwd - attention inside the kept blocks (section 2.2,
