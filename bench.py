@@ -141,13 +141,25 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device="cuda") -> float:
+    """The largest of the ranks' values (every rank gets it). The only
+    collective besides the barrier: the data path exchanges nothing."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(w: "li.Workload", rank: int) -> "li.Workload":
+    """Rank r streams its own video: the same shapes, seed + 1000 r (weak scaling)."""
+    return li.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+
+
+def whole_job_ms_per_chunk(step_ms_max: float, chunks_per_rank_step: int, world: int) -> float:
+    """All ranks process their chunks side by side in the slowest rank's step time."""
+    return step_ms_max / (chunks_per_rank_step * world)
 
 
 def attn_flops(blk_cnt: torch.Tensor, blk_idx: torch.Tensor, cache, Hb: int, Wb: int, D: int,
@@ -174,7 +186,7 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     peaks = load_peaks()
     # each rank streams an independent video (weak scaling)
-    w = li.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+    w = rank_workload(w, rank)
     streaming = w.kv_past[0] > 0 or w.B > 1
     x = li.make_inputs(w)
     params = lc.SelectParams(top_k=w.top_k, density=w.density, window=w.window,
@@ -206,10 +218,10 @@ def run_ours(args, world, rank, local):
             step.cache.set_state(base_state)
             if ev is not None:
                 ev[0].record()
-            lc.pool_qk(q, k, step.q_pool, step.k_pool)
+            lc.pool_qk(q, None, step.q_pool)
             if ev is not None:
                 ev[1].record()
-            lc.kv_append(step.cache, k, v, step.k_pool)
+            lc.kv_append(step.cache, k, v)  # pools K while copying it
             if ev is not None:
                 ev[2].record()
             lc.select_blocks(step.q_pool, step.q_frames, step.cache, step.params, step.kmax,
@@ -304,7 +316,7 @@ def run_ours(args, world, rank, local):
     mean_step = statistics.mean(step_ms)
     mean_step_max = max_over_ranks(mean_step, world)
     chunks_per_step = CHUNKS_PER_STEP.get(args.workload, 1) * w.B
-    value = mean_step_max / (chunks_per_step * world)
+    value = whole_job_ms_per_chunk(mean_step_max, chunks_per_step, world)
 
     flops = attn_flops(sel_ref.blk_cnt, sel_ref.blk_idx, cache, w.Hb, w.Wb, w.D)
     attn_s = per_kernel["attn"] / 1e3
@@ -336,7 +348,7 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(e_start, e_end))
         e2e_ms = max_over_ranks(e2e_ms, world)
-        e2e = {"value": e2e_ms / (chunks_per_step * world), "unit": UNIT,
+        e2e = {"value": whole_job_ms_per_chunk(e2e_ms, chunks_per_step, world), "unit": UNIT,
                "h2d_bytes_per_step": hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2,
                "d2h_bytes_per_step": ho.numel() * 2}
     else:
@@ -358,7 +370,7 @@ def run_ours(args, world, rank, local):
                 e_end[i - args.warmup].record()
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(e_start, e_end)), world)
-        e2e = {"value": e2e_ms / (chunks_per_step * world), "unit": UNIT,
+        e2e = {"value": whole_job_ms_per_chunk(e2e_ms, chunks_per_step, world), "unit": UNIT,
                "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel()) * 2,
                "d2h_bytes_per_step": ho.numel() * 2}
     if lc.last_device_error() != 0:
@@ -366,12 +378,18 @@ def run_ours(args, world, rank, local):
 
     # HBM-side kernels: algorithmic bytes per launch
     tokens_q = w.B * w.H * q_frames_step * w.Y * w.X
-    # pool reads Q and the new K (bf16) once and writes one float64 row per block
-    bytes_pool = 2 * tokens_q * w.D * 2 + 2 * (tokens_q // 128) * w.D * 8
-    hbm = {"pool_gbs": bytes_pool / (per_kernel["pool"] / 1e3) / 1e9}
     if "kv_append" in per_kernel:
-        bytes_app = 2 * (2 * tokens_q * w.D * 2) + 2 * (tokens_q // 128) * w.D * 8
-        hbm["kv_append_gbs"] = bytes_app / (per_kernel["kv_append"] / 1e3) / 1e9
+        # pool reads Q (bf16) once and writes one float64 row per block; the
+        # append reads the new K and V once, writes them into the ring and
+        # writes K's pooled rows
+        bytes_pool = tokens_q * w.D * 2 + (tokens_q // 128) * w.D * 8
+        bytes_app = 2 * (2 * tokens_q * w.D * 2) + (tokens_q // 128) * w.D * 8
+        hbm = {"pool_gbs": bytes_pool / (per_kernel["pool"] / 1e3) / 1e9,
+               "kv_append_gbs": bytes_app / (per_kernel["kv_append"] / 1e3) / 1e9}
+    else:
+        # whole clip: pool reads Q and K once and writes their pooled rows
+        bytes_pool = 2 * tokens_q * w.D * 2 + 2 * (tokens_q // 128) * w.D * 8
+        hbm = {"pool_gbs": bytes_pool / (per_kernel["pool"] / 1e3) / 1e9}
 
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "attn_fwd_%s.traffic.txt" % args.workload)

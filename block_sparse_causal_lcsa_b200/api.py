@@ -131,14 +131,17 @@ class KVCache:
             self.struct.end[b] = hi
 
 
-def kv_append(cache: KVCache, k_new: torch.Tensor, v_new: torch.Tensor, k_pool_new: torch.Tensor,
-              stream_offset: int = 0, stream: Optional[torch.cuda.Stream] = None) -> None:
-    """Append a chunk (and its pooled K) to streams [offset, offset+B) of the cache."""
+def kv_append(cache: KVCache, k_new: torch.Tensor, v_new: torch.Tensor,
+              k_pool_new: Optional[torch.Tensor] = None, stream_offset: int = 0,
+              stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Append a chunk to streams [offset, offset+B) of the cache. Without
+    k_pool_new the call pools K itself while copying it (one read of K)."""
     kd, vd = tensor_desc(k_new), tensor_desc(v_new)
-    if not k_pool_new.is_contiguous() or k_pool_new.dtype != torch.float64:
+    if k_pool_new is not None and (not k_pool_new.is_contiguous() or k_pool_new.dtype != torch.float64):
         raise ValueError("k_pool_new must be contiguous float64")
     _check(_lib.lcsa_kv_append(C.byref(cache.struct), C.byref(kd), C.byref(vd),
-                               k_pool_new.data_ptr(), stream_offset, _stream(stream)),
+                               k_pool_new.data_ptr() if k_pool_new is not None else None,
+                               stream_offset, _stream(stream)),
            "lcsa_kv_append")
 
 
@@ -253,24 +256,21 @@ def debug_set_wait_limit_ns(ns: int) -> None:
 
 
 class StreamingStep:
-    """One streaming LCSA step over preallocated buffers: pool Q and the new K,
-    append K/V and pooled K to the cache, select the top-K blocks, attend.
+    """One streaming LCSA step over preallocated buffers: pool Q, append K/V to
+    the cache (pooling K on the way), select the top-K blocks, attend.
 
     The four library calls are the whole step; buffers are allocated once here
     so that repeated steps launch kernels only.
     """
 
-    def __init__(self, cache: KVCache, q_frames: int, params: SelectParams, new_frames: int = None):
+    def __init__(self, cache: KVCache, q_frames: int, params: SelectParams):
         self.cache = cache
         self.q_frames = q_frames
         self.params = params
         dev = cache.k.device
         B, H, Y, X, D = cache.B, cache.H, cache.Y, cache.X, cache.D
-        nf = q_frames if new_frames is None else new_frames
         nQT = (q_frames + 1) // 2
         self.q_pool = torch.empty((B, H, nQT, Y // 8, X // 8, D), dtype=torch.float64, device=dev)
-        self.k_pool = torch.empty((B, H, (nf + 1) // 2, Y // 8, X // 8, D), dtype=torch.float64,
-                                  device=dev)
         # capacity for the fullest cache state this step can see
         full = _abi.KVCacheStruct.from_buffer_copy(cache.struct)
         for b in range(B):
@@ -287,8 +287,8 @@ class StreamingStep:
 
     def __call__(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
                  stream: Optional[torch.cuda.Stream] = None):
-        pool_qk(q, k_new, self.q_pool, self.k_pool, stream)
-        kv_append(self.cache, k_new, v_new, self.k_pool, 0, stream)
+        pool_qk(q, None, self.q_pool, None, stream)
+        kv_append(self.cache, k_new, v_new, None, 0, stream)
         select_blocks(self.q_pool, self.q_frames, self.cache, self.params, self.kmax,
                       self.blk_idx, self.blk_cnt, self.workspace, stream)
         sparse_attn_fwd(q, self.cache, self.blk_idx, self.blk_cnt, self.o, self.lse, stream=stream)

@@ -13,7 +13,7 @@
 #include "lcsa.h"
 #include "attn_fwd.cuh"
 #include "kv_append.cuh"
-#include "pool.cuh"
+#include "ingest.cuh"
 #include "select.cuh"
 
 // Scratch of lcsa_select_blocks_noalloc: the score keys that the caller's
@@ -176,6 +176,24 @@ int32_t kmax_for(int nKT, int nQT, int Hb, int Wb, const lcsa_select_params* p) 
   return K < C ? K : C;
 }
 
+void set_ingest_source(IngestTensor& it, const lcsa_tensor* t) {
+  it.src = static_cast<const __nv_bfloat16*>(t->data);
+  it.sb = t->stride_b; it.sh = t->stride_h; it.st = t->stride_t;
+  it.sy = t->stride_y; it.sx = t->stride_x;
+  it.T = t->T;
+  it.nT = temporal_blocks(t->T);
+}
+
+// One CTA per block of every tensor of p (a tensor with 0 units is skipped).
+lcsa_status launch_ingest(const IngestParams& p, int D, cudaStream_t cs) {
+  const int64_t grid = p.t[0].units + p.t[1].units + p.t[2].units;
+  if (grid > 0x7fffffff) return LCSA_ERR_SHAPE;
+  if (grid == 0) return LCSA_OK;
+  if (D == 128) ingest_kernel<128><<<static_cast<unsigned>(grid), INGEST_THREADS, 0, cs>>>(p);
+  else ingest_kernel<64><<<static_cast<unsigned>(grid), INGEST_THREADS, 0, cs>>>(p);
+  return launched();
+}
+
 }  // namespace
 }  // namespace lcsa
 
@@ -214,29 +232,22 @@ lcsa_status lcsa_pool_qk(const lcsa_tensor* q, const lcsa_tensor* k, double* q_p
   int dev;
   unsigned int* err;
   if ((s = device_setup(&dev, &err)) != LCSA_OK) return s;
-  PoolParams p{};
-  p.H = q->H;
+  IngestParams p{};
+  p.H = q->H; p.Y = q->Y; p.X = q->X;
   p.Hb = q->Y / 8;
   p.Wb = q->X / 8;
+  p.cap = 2;  // no ring destination
   const lcsa_tensor* ts[2] = {q, k};
   double* outs[2] = {q_pool, k_pool};
   for (int i = 0; i < 2; ++i) {
-    PoolTensor& pt = p.t[i];
-    if (ts[i] == nullptr) { pt.units = 0; continue; }
-    pt.data = static_cast<const __nv_bfloat16*>(ts[i]->data);
-    pt.out = outs[i];
-    pt.sb = ts[i]->stride_b; pt.sh = ts[i]->stride_h; pt.st = ts[i]->stride_t;
-    pt.sy = ts[i]->stride_y; pt.sx = ts[i]->stride_x;
-    pt.T = ts[i]->T;
-    pt.nT = temporal_blocks(ts[i]->T);
-    pt.units = static_cast<int64_t>(ts[i]->B) * ts[i]->H * pt.nT * p.Hb * p.Wb;
+    IngestTensor& it = p.t[i];
+    if (ts[i] == nullptr) continue;  // units 0
+    set_ingest_source(it, ts[i]);
+    it.tb_first = 0;
+    it.units = static_cast<int64_t>(ts[i]->B) * ts[i]->H * it.nT * p.Hb * p.Wb;
+    it.pool_out = outs[i];
   }
-  const int64_t grid = p.t[0].units + p.t[1].units;  // one CTA per block
-  if (grid > 0x7fffffff) return LCSA_ERR_SHAPE;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (q->D == 128) pool_kernel<128><<<static_cast<unsigned>(grid), POOL_THREADS, 0, cs>>>(p);
-  else pool_kernel<64><<<static_cast<unsigned>(grid), POOL_THREADS, 0, cs>>>(p);
-  return launched();
+  return launch_ingest(p, q->D, static_cast<cudaStream_t>(stream));
 }
 
 lcsa_status lcsa_kv_append(lcsa_kv_cache* kv, const lcsa_tensor* k_new, const lcsa_tensor* v_new,
@@ -244,8 +255,7 @@ lcsa_status lcsa_kv_append(lcsa_kv_cache* kv, const lcsa_tensor* k_new, const lc
   lcsa_status s = check_cache(kv);
   if (s != LCSA_OK) return s;
   if ((s = check_tensor(k_new)) != LCSA_OK || (s = check_tensor(v_new)) != LCSA_OK) return s;
-  if (k_pool_new == nullptr) return LCSA_ERR_INVALID_ARG;
-  if (!aligned16(k_pool_new)) return LCSA_ERR_ALIGN;
+  if (k_pool_new != nullptr && !aligned16(k_pool_new)) return LCSA_ERR_ALIGN;
   const lcsa_tensor* kn = k_new;
   if (v_new->B != kn->B || v_new->H != kn->H || v_new->T != kn->T || v_new->Y != kn->Y ||
       v_new->X != kn->X || v_new->D != kn->D)
@@ -276,6 +286,32 @@ lcsa_status lcsa_kv_append(lcsa_kv_cache* kv, const lcsa_tensor* k_new, const lc
   int dev;
   unsigned int* err;
   if ((s = device_setup(&dev, &err)) != LCSA_OK) return s;
+  if (k_pool_new == nullptr) {
+    // pool K while copying it: one read of K and V, one CTA per block
+    IngestParams ip{};
+    ip.H = kn->H; ip.Y = kn->Y; ip.X = kn->X;
+    ip.Hb = kn->Y / 8; ip.Wb = kn->X / 8;
+    ip.cap = cap;
+    ip.stream_offset = stream_offset;
+    for (int bn = 0; bn < kn->B; ++bn) ip.first_abs[bn] = p.first_abs[bn];
+    const lcsa_tensor* ts[2] = {kn, v_new};
+    __nv_bfloat16* dsts[2] = {static_cast<__nv_bfloat16*>(kv->k), static_cast<__nv_bfloat16*>(kv->v)};
+    for (int i = 0; i < 2; ++i) {
+      IngestTensor& it = ip.t[i];
+      set_ingest_source(it, ts[i]);
+      it.tb_first = nTn - copy_blocks;
+      it.units = static_cast<int64_t>(kn->B) * kn->H * copy_blocks * ip.Hb * ip.Wb;
+      it.copy_dst = dsts[i];
+    }
+    ip.t[0].pool_out = kv->k_pool;
+    ip.t[0].pool_ring = 1;
+    if ((s = launch_ingest(ip, kn->D, static_cast<cudaStream_t>(stream))) != LCSA_OK) return s;
+    for (int bn = 0; bn < kn->B; ++bn) {
+      kv->begin[bn + stream_offset] = new_begin[bn];
+      kv->end[bn + stream_offset] = new_end[bn];
+    }
+    return LCSA_OK;
+  }
   p.k_new = static_cast<const __nv_bfloat16*>(kn->data);
   p.v_new = static_cast<const __nv_bfloat16*>(v_new->data);
   p.kp_new = k_pool_new;
@@ -472,8 +508,9 @@ lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_cache* kv, 
   p.wait_limit_ns = g_wait_limit_ns;
   p.err = err;
   for (int b = 0; b < kv->B; ++b) { p.kv_begin[b] = kv->begin[b]; p.kv_end[b] = kv->end[b]; }
-  const int64_t grid = static_cast<int64_t>(q->B) * q->H * p.nQB;
+  const int64_t grid = static_cast<int64_t>(q->B) * q->H * p.nQB;  // one CTA per query block
   if (grid > 0x7fffffff) return LCSA_ERR_SHAPE;
+  if (grid == 0) return LCSA_OK;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (q->D == 128)
     attn_fwd_kernel<128><<<static_cast<unsigned>(grid), ATTN_THREADS, AttnLayout<128>::SMEM_BYTES, cs>>>(tq, tk, tv, p);

@@ -9,8 +9,9 @@
  * sparse attention"). One streaming step is four calls, all asynchronous on
  * the caller's CUDA stream:
  *
- *   lcsa_pool_qk        mean-pool Q and K over 2x8x8 (t,y,x) token blocks
+ *   lcsa_pool_qk        mean-pool Q (and K) over 2x8x8 (t,y,x) token blocks
  *   lcsa_kv_append      write the chunk's K, V and pooled K into the ring cache
+ *                       (pooling K on the way when no pooled K is given)
  *   lcsa_select_blocks  coarse block scores + causal/window masks + top-K
  *   lcsa_sparse_attn_fwd  online-softmax attention over the kept blocks
  *
@@ -167,7 +168,9 @@ LCSA_API lcsa_status lcsa_pool_qk(const lcsa_tensor* q, const lcsa_tensor* k,
  * k_new, v_new  token tensors [Bn][H][Tn][Y][X][D] with the cache's H, Y, X,
  *             D; they fill cache streams [stream_offset, stream_offset+Bn).
  * k_pool_new  device, float64 [Bn][H][ceil(Tn/2)][Y/8][X/8][D], the pooled
- *             K of the chunk (lcsa_pool_qk on k_new).
+ *             K of the chunk (lcsa_pool_qk on k_new), or NULL: the call then
+ *             pools k_new itself while copying it (one HBM read of K for both;
+ *             the same float64 means lcsa_pool_qk gives).
  * Tn must be even, except for the first chunk of an empty stream, whose
  * frames are then placed so that the oldest block holds one frame. Only the
  * newest cap_frames frames of a chunk longer than the cache are written.

@@ -201,6 +201,37 @@ def test_odd_first_chunk_partial_blocks(lc, first, q_frames):
         check_output(o[0, h].double().cpu().numpy(), ref["O"], lse[0, h].double().cpu().numpy(), ref["LSE"])
 
 
+@pytest.mark.parametrize("cap,chunks", [(8, (3, 2, 2, 2, 2)), (4, (5, 2, 6)), (6, (2, 10, 2)),
+                                         (6, (1, 2, 2, 2))])
+def test_fused_append_equals_pool_then_append(lc, cap, chunks):
+    """kv_append without a pooled K (K pooled while it is copied) leaves the
+    ring cache bit for bit as pool_qk followed by kv_append with the pooled K:
+    odd first chunks, chunks longer than the cache, wrap-around."""
+    H, Y, X, D = 2, 16, 24, 128
+    g = torch.Generator().manual_seed(81 + cap)
+    a = lc.KVCache(2, H, cap, Y, X, D)
+    b = lc.KVCache(2, H, cap, Y, X, D)
+    for c in (a, b):
+        c.k.zero_(), c.v.zero_(), c.k_pool.zero_()
+    for t in chunks:
+        k = (torch.randn((2, H, t, Y, X, D), generator=g) * 3).to(torch.bfloat16).cuda()
+        v = torch.randn((2, H, t, Y, X, D), generator=g).to(torch.bfloat16).cuda()
+        lc.kv_append(a, k, v)
+        lc.kv_append(b, k, v, lc.pool_qk(k)[0])
+        assert a.state() == b.state()
+    torch.cuda.synchronize()
+    assert lc.last_device_error() == 0
+    assert torch.equal(a.k, b.k) and torch.equal(a.v, b.v)
+    assert torch.equal(a.k_pool, b.k_pool)
+    # and the pooled rows are the oracle's means of the cached frames
+    for s_ in range(2):
+        for h in range(H):
+            lo, hi = a.state()[s_]
+            frames = torch.stack([a.k[s_, h, f % cap].cpu() for f in range(lo, hi)])
+            ref = orc.pool_blocks(orc.widen(frames))
+            assert np.array_equal(ring_to_logical(a, a.k_pool.cpu().numpy(), s_, h), ref)
+
+
 @pytest.mark.parametrize("kw", [dict(density=1.0), dict(top_k=1000), dict(top_k=1),
                                 dict(density=0.3, window=99, window_mode=1)])
 def test_degenerate_selection_parameters(lc, kw):
