@@ -18,7 +18,8 @@ cache, section 2.3 "locality-constrained sparse attention"):
    boundary-preserve rule (``allowed_blocks``).
 3. Only the top-K key blocks per query block are kept (``select_row``).
 4. Full softmax attention runs over the tokens of the kept blocks
-   (``attend_rows``).
+   (``attend_rows``); its gradients for training follow by the chain rule
+   with the selection held fixed (``attend_rows_backward``).
 5. The streaming KV cache appends each chunk and drops the oldest frames
    (``kv_append``).
 
@@ -29,7 +30,9 @@ the window rules, the K rule and the tie rule) are stated on each function.
 Pins (checked in ``tests/test_oracle_pins.py`` against things other than this
 file): exact rational means, brute-force top-K, hand-derived golden cases,
 full-density equality with masked dense attention from torch, unit row sums,
-the single-block textbook case, window invariants. Parity with the authors'
+the single-block textbook case, window invariants; for the gradients: central
+finite differences, torch autograd of masked dense attention, and the closed
+forms sum_t dk_t = 0, sum_t dv_t = sum_r do_r, dq = dk = 0 for equal values. Parity with the authors'
 own implementation is unpinned: the pages print no numeric example of it.
 """
 from __future__ import annotations
@@ -232,6 +235,71 @@ def gather_blocks(x: np.ndarray, ids: Sequence[int]) -> np.ndarray:
         yb, xb = divmod(r, Wb)
         parts.append(block_token_view(x, tb[t], yb, xb))
     return np.concatenate(parts, axis=0)
+
+
+# --------------------------------------------------------------------------- #
+# 4b. Gradients of the attention over the kept blocks. The pages train stage 2
+#     (and stage 3) with the block-sparse causal mask (section 2.2, stage 2:
+#     "trained with the flow-matching loss"), so the attention needs its
+#     backward pass. The selection is a constant mask: the top-K of pooled
+#     scores is piecewise constant, its derivative is zero almost everywhere.
+# --------------------------------------------------------------------------- #
+def attend_rows_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray,
+                         do: np.ndarray) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Gradients of O = softmax(q k^T / sqrt(d)) v with respect to q, k, v for
+    the output gradient ``do``, by the chain rule through the row softmax:
+
+        P = softmax(S), S = q k^T / sqrt(d), O = P v
+        dV = P^T dO,  dP = dO v^T,  delta_r = sum_d dO_rd O_rd (= sum_t P_rt dP_rt)
+        dS = P * (dP - delta),  dq = dS k / sqrt(d),  dk = dS^T q / sqrt(d)
+    """
+    scale = 1.0 / math.sqrt(q.shape[1])
+    s = (q @ k.T) * scale
+    e = np.exp(s - s.max(axis=1, keepdims=True))
+    p = e / e.sum(axis=1, keepdims=True)
+    o = p @ v
+    dv = p.T @ do
+    dp = do @ v.T
+    delta = (do * o).sum(axis=1, keepdims=True)
+    ds = p * (dp - delta)
+    return (ds @ k) * scale, (ds.T @ q) * scale, dv
+
+
+def block_token_index(F: int, Y: int, X: int, ids: Sequence[int]) -> np.ndarray:
+    """Flat indices into [F][Y][X] of the tokens of the given blocks, in the
+    order ``gather_blocks`` concatenates them."""
+    _, Hb, Wb = block_grid(F, Y, X)
+    tb = temporal_blocks(F)
+    flat = np.arange(F * Y * X).reshape(F, Y, X)
+    parts = []
+    for j in ids:
+        t, r = divmod(int(j), Hb * Wb)
+        yb, xb = divmod(r, Wb)
+        parts.append(block_token_view(flat[..., None], tb[t], yb, xb)[:, 0])
+    return np.concatenate(parts)
+
+
+def attend_head_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, sel: Sequence[np.ndarray],
+                         do: np.ndarray):
+    """dq, dk, dv of one (stream, head): ``q``/``do`` [Tq][Y][X][D], ``k``/``v``
+    [F][Y][X][D], ``sel`` the kept key blocks of every query block. Each query
+    block's gradients come from ``attend_rows_backward`` over its kept tokens;
+    the key and value gradients of all query blocks are summed per token."""
+    Tq, Y, X, D = q.shape
+    F = k.shape[0]
+    nQT, Hb, Wb = block_grid(Tq, Y, X)
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape).reshape(-1, D)
+    dv = np.zeros(v.shape).reshape(-1, D)
+    kf, vf = k.reshape(-1, D), v.reshape(-1, D)
+    for i in range(nQT * Hb * Wb):
+        qidx = block_token_index(Tq, Y, X, [i])
+        kidx = block_token_index(F, Y, X, sel[i])
+        gq, gk, gv = attend_rows_backward(q.reshape(-1, D)[qidx], kf[kidx], vf[kidx], do.reshape(-1, D)[qidx])
+        dq.reshape(-1, D)[qidx] = gq
+        np.add.at(dk, kidx, gk)
+        np.add.at(dv, kidx, gv)
+    return dq, dk.reshape(k.shape), dv.reshape(v.shape)
 
 
 # --------------------------------------------------------------------------- #
