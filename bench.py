@@ -429,6 +429,105 @@ def run_ours(args, world, rank, local):
 
 
 # ----------------------------------------------------------------------------- oracle arm
+def run_backward(args, world, rank, local):
+    """Attention gradients for training with the block-sparse causal mask: the
+    whole clip is the key timeline, the forward runs once (untimed), then each
+    step is one lcsa_sparse_attn_bwd call (prep, transposed lists, dQ, dK/dV)."""
+    import block_sparse_causal_lcsa_b200 as lc
+
+    w = rank_workload(li.workload(args.workload), rank)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    x = li.make_inputs(w)
+    cache = lc.KVCache(w.B, w.H, w.cap_frames, w.Y, w.X, w.D, device=dev)
+    for b in range(w.B):
+        kb = x["k"][b].unsqueeze(0).to(dev)
+        vb = x["v"][b].unsqueeze(0).to(dev)
+        lc.kv_append(cache, kb, vb, stream_offset=b)
+    q = x["q"].to(dev)
+    params = lc.SelectParams(top_k=w.top_k, density=w.density, window=w.window, window_mode=w.window_mode)
+    idx, cnt = lc.select_blocks(lc.pool_qk(q)[0], w.q_frames, cache, params)
+    o, lse = lc.sparse_attn_fwd(q, cache, idx, cnt)
+    g = torch.Generator().manual_seed(w.seed + 11)
+    d_o = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(dev)
+    dq, dk, dv = torch.empty_like(q), torch.zeros_like(cache.k), torch.zeros_like(cache.v)
+    ws = torch.empty(max(lc.sparse_attn_bwd_workspace_bytes(cache, w.q_frames), 16), dtype=torch.uint8, device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        lc.sparse_attn_bwd(q, cache, idx, cnt, o, lse, d_o, dq, dk, dv, ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if lc.last_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for a, b in evs:
+        flush.zero_()
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    time.sleep(0.2)
+    clk = clocks.stop()
+    if lc.last_device_error() != 0:
+        raise RuntimeError("device error during the timed steps")
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world)
+    fwd_flops = attn_flops(cnt, idx, cache, w.Hb, w.Wb, w.D)
+    algo_flops = 2.5 * fwd_flops        # dS/dP, dQ, dK, dV and the recomputed S: 5 products
+    exec_flops = 3.5 * fwd_flops        # this implementation: S and dP in both kernels, 7 products
+    achieved = algo_flops / (ms / 1e3) / 1e12
+    line = {
+        "metric": "ms per attention backward of a 101-frame 768x1408 clip (training, block-sparse causal)",
+        "value": round(ms / world, 4), "unit": "ms/clip", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, shapes of the pages' clip workload)",
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload, "mode": "backward",
+                   "l2": "flushed before every timed step (512 MB write)"},
+        "roofline": {"bound": "tensor", "kernel": "attention backward (4 launches)", "achieved": round(achieved, 2),
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "peak_source": "measured bf16 burst (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
+                     else "fallback", "flops_algorithmic": algo_flops, "flops_executed": exec_flops,
+                     "executed_tflops": round(exec_flops / (ms / 1e3) / 1e12, 2), "traffic": None},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import lcsa_oracle as orc
+        t0 = time.perf_counter()
+        h = 0
+        qh, kh, vh = orc.widen(x["q"][0, h]), orc.widen(x["k"][0][h]), orc.widen(x["v"][0][h])
+        sel = [idx[0, h, i, :int(cnt[0, h, i])].cpu().numpy() for i in range(cnt.shape[2])]
+        # a bounded sample: the first query blocks of one head, scaled by their share of the kept pairs
+        n_rows = 0
+        kept = 0
+        Tq, Y, X, D = qh.shape
+        for i in range(len(sel)):
+            qidx = orc.block_token_index(Tq, Y, X, [i])
+            kidx = orc.block_token_index(kh.shape[0], Y, X, sel[i])
+            orc.attend_rows_backward(qh.reshape(-1, D)[qidx], kh.reshape(-1, D)[kidx], vh.reshape(-1, D)[kidx],
+                                     orc.widen(d_o[0, h].cpu()).reshape(-1, D)[qidx])
+            n_rows += 1
+            kept += len(sel[i])
+            if time.perf_counter() - t0 > args.cpu_budget:
+                break
+        el = time.perf_counter() - t0
+        total_kept = int(cnt.sum().item())
+        cpu_ms = el / kept * total_kept * 1e3
+        line["cpu_baseline"] = {"value": round(cpu_ms, 1), "unit": "ms/clip", "cores": _threads(), "kind": "oracle",
+                                "sample": "%d query blocks (%d kept block pairs) of head 0, attend_rows_backward "
+                                          "in fp64, scaled by kept pairs to all %d" % (n_rows, kept, total_kept)}
+    return line
+
+
 def _threads():
     try:
         from threadpoolctl import threadpool_info
@@ -500,6 +599,8 @@ def main():
     ap.add_argument("--workload", default="chunk", choices=sorted(WORKLOAD_TEXT))
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="fwd", choices=["fwd", "bwd"],
+                    help="fwd: the streaming step (default); bwd: the attention backward on a clip")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -512,7 +613,12 @@ def main():
         return
     world, rank, local = dist_setup(args.gpus)
     try:
-        line = run_ours(args, world, rank, local)
+        if args.mode == "bwd":
+            if args.workload == "chunk":
+                args.workload = "clip"
+            line = run_backward(args, world, rank, local)
+        else:
+            line = run_ours(args, world, rank, local)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

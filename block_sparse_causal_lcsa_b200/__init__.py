@@ -22,6 +22,8 @@ from .api import (  # noqa: F401
     select_blocks_noalloc,
     select_kmax,
     select_workspace_bytes,
+    sparse_attn_bwd,
+    sparse_attn_bwd_workspace_bytes,
     sparse_attn_fwd,
     tensor_desc,
 )

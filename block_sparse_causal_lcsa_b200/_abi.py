@@ -76,6 +76,11 @@ PROTOTYPES = {
     "lcsa_sparse_attn_fwd": (C.c_int, [C.POINTER(Tensor), C.POINTER(KVCacheStruct), C.c_void_p,
                                        C.c_void_p, C.c_int32, C.POINTER(Tensor), C.c_void_p,
                                        C.c_void_p]),
+    "lcsa_sparse_attn_bwd_workspace_bytes": (C.c_size_t, [C.POINTER(KVCacheStruct), C.c_int32]),
+    "lcsa_sparse_attn_bwd": (C.c_int, [C.POINTER(Tensor), C.POINTER(KVCacheStruct), C.c_void_p, C.c_void_p,
+                                       C.c_int32, C.POINTER(Tensor), C.c_void_p, C.POINTER(Tensor),
+                                       C.POINTER(Tensor), C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t,
+                                       C.c_void_p]),
     "lcsa_last_device_error": (C.c_int, [C.c_void_p]),
     "lcsa_debug_set_wait_limit_ns": (C.c_int, [C.c_uint64]),
     "lcsa_debug_stalled_wait": (C.c_int, [C.c_uint64, C.c_void_p]),

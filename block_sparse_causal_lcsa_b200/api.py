@@ -232,6 +232,39 @@ def sparse_attn_fwd(q: torch.Tensor, cache: KVCache, blk_idx: torch.Tensor, blk_
     return o, lse
 
 
+def sparse_attn_bwd_workspace_bytes(cache: KVCache, q_frames: int) -> int:
+    return int(_lib.lcsa_sparse_attn_bwd_workspace_bytes(C.byref(cache.struct), q_frames))
+
+
+def sparse_attn_bwd(q: torch.Tensor, cache: KVCache, blk_idx: torch.Tensor, blk_cnt: torch.Tensor,
+                    o: torch.Tensor, lse: torch.Tensor, d_o: torch.Tensor,
+                    dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+                    dv: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None):
+    """Gradients of sparse_attn_fwd for the same selection: (dq like q, dk and
+    dv in the cache layout [B][H][cap][Y][X][D]). dk / dv default to zeros, so
+    ring slots outside the cached frames read as zero."""
+    if dq is None:
+        dq = torch.empty_like(q)
+    if dk is None:
+        dk = torch.zeros_like(cache.k)
+    if dv is None:
+        dv = torch.zeros_like(cache.v)
+    need = sparse_attn_bwd_workspace_bytes(cache, q.shape[2])
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    for t in (blk_idx, blk_cnt, lse, dk, dv):
+        if not t.is_contiguous():
+            raise ValueError("blk_idx, blk_cnt, lse, dk and dv must be contiguous")
+    qd, od, gd, dqd = tensor_desc(q), tensor_desc(o), tensor_desc(d_o), tensor_desc(dq)
+    _check(_lib.lcsa_sparse_attn_bwd(C.byref(qd), C.byref(cache.struct), blk_idx.data_ptr(), blk_cnt.data_ptr(),
+                                     blk_idx.shape[-1], C.byref(od), lse.data_ptr(), C.byref(gd), C.byref(dqd),
+                                     dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                                     workspace.numel() * workspace.element_size(), _stream(stream)),
+           "lcsa_sparse_attn_bwd")
+    return dq, dk, dv
+
+
 def last_device_error(stream: Optional[torch.cuda.Stream] = None) -> int:
     """Synchronise the stream, read and clear the device error word (status code)."""
     return int(_lib.lcsa_last_device_error(_stream(stream)))

@@ -12,6 +12,7 @@
 
 #include "lcsa.h"
 #include "attn_fwd.cuh"
+#include "attn_bwd.cuh"
 #include "kv_append.cuh"
 #include "ingest.cuh"
 #include "select.cuh"
@@ -61,7 +62,15 @@ lcsa_status device_setup(int* dev_out, unsigned int** err_out) {
         cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(score_smem_bytes(128))) != cudaSuccess ||
         cudaFuncSetAttribute(score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(score_smem_bytes(64))) != cudaSuccess)
+                             static_cast<int>(score_smem_bytes(64))) != cudaSuccess ||
+        cudaFuncSetAttribute(bwd_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             BwdLayout<128>::SMEM_DQ) != cudaSuccess ||
+        cudaFuncSetAttribute(bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             BwdLayout<64>::SMEM_DQ) != cudaSuccess ||
+        cudaFuncSetAttribute(bwd_dkdv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             BwdLayout<128>::SMEM_KV) != cudaSuccess ||
+        cudaFuncSetAttribute(bwd_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             BwdLayout<64>::SMEM_KV) != cudaSuccess)
       return LCSA_ERR_CUDA;
     g_attr_done[dev] = true;
   }
@@ -432,6 +441,127 @@ lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames, const lcs
   const unsigned tthreads = static_cast<unsigned>(((c_stride + slots - 1) / slots + 31) / 32 * 32);
   if (slots == 1) topk_kernel<1><<<static_cast<unsigned>(rows), tthreads, 0, cs>>>(p);
   else topk_kernel<2><<<static_cast<unsigned>(rows), tthreads, 0, cs>>>(p);
+  return launched();
+}
+
+// Backward workspace: LSE*log2(e) and delta per query row in block order,
+// then the per-key-block count and list of the query blocks that kept it.
+struct BwdSizes {
+  int64_t BH, nQB, nKBmax, off_delta, off_cnt, off_list, total;
+};
+static BwdSizes bwd_sizes(const lcsa_kv_cache* kv, int32_t q_frames) {
+  BwdSizes z{};
+  const int64_t HbWb = static_cast<int64_t>(kv->Y / 8) * (kv->X / 8);
+  int nKT = 0;
+  for (int b = 0; b < kv->B; ++b) {
+    const int n = static_cast<int>((kv->end[b] >> 1) - (kv->begin[b] >> 1));
+    nKT = n > nKT ? n : nKT;
+  }
+  z.BH = static_cast<int64_t>(kv->B) * kv->H;
+  z.nQB = temporal_blocks(q_frames) * HbWb;
+  z.nKBmax = nKT * HbWb;
+  const int64_t vec = z.BH * z.nQB * 128 * 4;
+  z.off_delta = vec;
+  z.off_cnt = 2 * vec;
+  z.off_list = z.off_cnt + (z.BH * z.nKBmax * 4 + 15) / 16 * 16;
+  z.total = z.off_list + z.BH * z.nKBmax * z.nQB * 4;
+  return z;
+}
+
+size_t lcsa_sparse_attn_bwd_workspace_bytes(const lcsa_kv_cache* kv, int32_t q_frames) {
+  if (kv == nullptr || q_frames < 1 || kv->B < 1 || kv->B > LCSA_MAX_STREAMS || kv->Y < 8 || kv->X < 8)
+    return 0;
+  return static_cast<size_t>(bwd_sizes(kv, q_frames).total);
+}
+
+lcsa_status lcsa_sparse_attn_bwd(const lcsa_tensor* q, const lcsa_kv_cache* kv, const int32_t* blk_idx,
+                                 const int32_t* blk_cnt, int32_t kmax, const lcsa_tensor* o, const float* lse,
+                                 const lcsa_tensor* d_o, lcsa_tensor* dq, void* dk, void* dv, void* workspace,
+                                 size_t workspace_bytes, lcsa_stream_t stream) {
+  lcsa_status s = check_tensor(q);
+  if (s != LCSA_OK) return s;
+  if ((s = check_cache(kv)) != LCSA_OK) return s;
+  if (o == nullptr || d_o == nullptr || dq == nullptr) return LCSA_ERR_INVALID_ARG;
+  if ((s = check_tensor(o)) != LCSA_OK || (s = check_tensor(d_o)) != LCSA_OK || (s = check_tensor(dq)) != LCSA_OK)
+    return s;
+  if (blk_idx == nullptr || blk_cnt == nullptr || kmax < 1 || lse == nullptr || dk == nullptr || dv == nullptr ||
+      workspace == nullptr)
+    return LCSA_ERR_INVALID_ARG;
+  if (q->B != kv->B || q->H != kv->H || q->Y != kv->Y || q->X != kv->X || q->D != kv->D) return LCSA_ERR_SHAPE;
+  const lcsa_tensor* like_q[3] = {o, d_o, dq};
+  for (const lcsa_tensor* t : like_q)
+    if (t->B != q->B || t->H != q->H || t->T != q->T || t->Y != q->Y || t->X != q->X || t->D != q->D)
+      return LCSA_ERR_SHAPE;
+  for (int b = 0; b < kv->B; ++b)
+    if (kv->end[b] - kv->begin[b] < q->T) return LCSA_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+    return LCSA_ERR_ALIGN;
+  const BwdSizes z = bwd_sizes(kv, q->T);
+  if (workspace_bytes < static_cast<size_t>(z.total)) return LCSA_ERR_WORKSPACE;
+  if (z.BH * z.nQB > 0x7fffffff || z.BH * z.nKBmax * 32 > 0x7fffffff) return LCSA_ERR_SHAPE;
+  int dev;
+  unsigned int* err;
+  if ((s = device_setup(&dev, &err)) != LCSA_OK) return s;
+  CUtensorMap tq, tdo, tk, tv;
+  const int64_t cs_x = kv->D, cs_y = static_cast<int64_t>(kv->X) * kv->D;
+  const int64_t cs_t = cs_y * kv->Y, cs_h = cs_t * kv->cap_frames;
+  if ((s = encode_map(&tq, q->data, q->B, q->H, q->T, q->Y, q->X, q->D, q->stride_h, q->stride_t, q->stride_y,
+                      q->stride_x)) != LCSA_OK ||
+      (s = encode_map(&tdo, d_o->data, q->B, q->H, q->T, q->Y, q->X, q->D, d_o->stride_h, d_o->stride_t,
+                      d_o->stride_y, d_o->stride_x)) != LCSA_OK ||
+      (s = encode_map(&tk, kv->k, kv->B, kv->H, kv->cap_frames, kv->Y, kv->X, kv->D, cs_h, cs_t, cs_y, cs_x)) !=
+          LCSA_OK ||
+      (s = encode_map(&tv, kv->v, kv->B, kv->H, kv->cap_frames, kv->Y, kv->X, kv->D, cs_h, cs_t, cs_y, cs_x)) !=
+          LCSA_OK)
+    return s;
+  BwdParams p{};
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.blk_idx = blk_idx;
+  p.blk_cnt = blk_cnt;
+  p.o = static_cast<const __nv_bfloat16*>(o->data);
+  p.d_o = static_cast<const __nv_bfloat16*>(d_o->data);
+  p.lse = lse;
+  p.dq = static_cast<__nv_bfloat16*>(dq->data);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.lse2_blk = reinterpret_cast<float*>(ws);
+  p.delta_blk = reinterpret_cast<float*>(ws + z.off_delta);
+  p.qcnt = reinterpret_cast<int32_t*>(ws + z.off_cnt);
+  p.qlist = reinterpret_cast<int32_t*>(ws + z.off_list);
+  p.osh = o->stride_h; p.ost = o->stride_t; p.osy = o->stride_y; p.osx = o->stride_x;
+  p.gsh = d_o->stride_h; p.gst = d_o->stride_t; p.gsy = d_o->stride_y; p.gsx = d_o->stride_x;
+  p.qsh = dq->stride_h; p.qst = dq->stride_t; p.qsy = dq->stride_y; p.qsx = dq->stride_x;
+  p.BH = static_cast<int32_t>(z.BH);
+  p.H = q->H; p.Tq = q->T; p.Y = q->Y; p.X = q->X; p.Hb = q->Y / 8; p.Wb = q->X / 8;
+  p.nQT = temporal_blocks(q->T);
+  p.nQB = static_cast<int32_t>(z.nQB);
+  p.kmax = kmax;
+  p.cap = kv->cap_frames;
+  p.nKBmax = static_cast<int32_t>(z.nKBmax);
+  p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(q->D)));
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(q->D)));
+  p.wait_limit_ns = g_wait_limit_ns;
+  p.err = err;
+  for (int b = 0; b < kv->B; ++b) { p.kv_begin[b] = kv->begin[b]; p.kv_end[b] = kv->end[b]; }
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const unsigned n_q = static_cast<unsigned>(z.BH * z.nQB), n_k = static_cast<unsigned>(z.BH * z.nKBmax);
+  if (q->D == 128) {
+    bwd_prep_kernel<128><<<n_q, 128, 0, cs>>>(p);
+  } else {
+    bwd_prep_kernel<64><<<n_q, 128, 0, cs>>>(p);
+  }
+  if ((s = launched()) != LCSA_OK) return s;
+  bwd_lists_kernel<<<static_cast<unsigned>((static_cast<int64_t>(n_k) * 32 + 255) / 256), 256, 0, cs>>>(p);
+  if ((s = launched()) != LCSA_OK) return s;
+  if (q->D == 128) {
+    bwd_dq_kernel<128><<<n_q, BWD_THREADS, BwdLayout<128>::SMEM_DQ, cs>>>(tq, tdo, tk, tv, p);
+    if ((s = launched()) != LCSA_OK) return s;
+    bwd_dkdv_kernel<128><<<n_k, BWD_THREADS, BwdLayout<128>::SMEM_KV, cs>>>(tq, tdo, tk, tv, p);
+  } else {
+    bwd_dq_kernel<64><<<n_q, BWD_THREADS, BwdLayout<64>::SMEM_DQ, cs>>>(tq, tdo, tk, tv, p);
+    if ((s = launched()) != LCSA_OK) return s;
+    bwd_dkdv_kernel<64><<<n_k, BWD_THREADS, BwdLayout<64>::SMEM_KV, cs>>>(tq, tdo, tk, tv, p);
+  }
   return launched();
 }
 

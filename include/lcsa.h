@@ -15,6 +15,8 @@
  *   lcsa_select_blocks  coarse block scores + causal/window masks + top-K
  *   lcsa_sparse_attn_fwd  online-softmax attention over the kept blocks
  *
+ * and, for training with the same mask, lcsa_sparse_attn_bwd (dQ, dK, dV).
+ *
  * Conventions
  * - Memory: the caller owns every buffer. The library allocates no device or
  *   host memory (the attention kernel allocates tensor memory on the SM for
@@ -283,6 +285,38 @@ LCSA_API lcsa_status lcsa_select_blocks_noalloc(const double* q_pool, int32_t q_
 LCSA_API lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_cache* kv,
                                  const int32_t* blk_idx, const int32_t* blk_cnt,
                                  int32_t kmax, lcsa_tensor* o, float* lse,
+                                 lcsa_stream_t stream);
+
+/*
+ * lcsa_sparse_attn_bwd - gradients of lcsa_sparse_attn_fwd for training with
+ * the block-sparse causal mask (section 2.2, stage 2: the model is adapted to
+ * block-sparse causal attention and trained with the flow-matching loss; stage
+ * 3 trains the one-step student with the same mask). The selection (blk_idx,
+ * blk_cnt, kmax, as passed to the forward) is held fixed.
+ *
+ * q, kv, blk_idx, blk_cnt, kmax  exactly as given to lcsa_sparse_attn_fwd.
+ * o, lse      the forward's output and log-sum-exp (lse required).
+ * d_o         token tensor like q: dLoss/dO.
+ * dq          token tensor like q (bf16), device: receives dLoss/dQ.
+ * dk, dv      device, bf16, contiguous in the cache layout
+ *             [B][H][cap_frames][Y][X][D]: every ring slot of a frame in
+ *             [begin, end) of each stream receives dLoss/dK, dLoss/dV (zero
+ *             for keys no query kept); other slots are not written.
+ * workspace   device scratch of at least lcsa_sparse_attn_bwd_workspace_bytes()
+ *             bytes, 16-byte aligned, owned by the caller.
+ * With P = exp(Q K^T / sqrt(D) - LSE), dP = dO V^T, delta = rowsum(dO * O) and
+ * dS = P (dP - delta): dQ = dS K / sqrt(D), dK = dS^T Q / sqrt(D), dV = P^T dO,
+ * summed over every query block that kept a key block. bf16 tensor-core
+ * products with float32 accumulation; P and dS rounded to bf16 before their
+ * products. Deterministic: no floating-point atomics. Errors as for the
+ * forward; LCSA_ERR_WORKSPACE if workspace_bytes is too small.
+ */
+LCSA_API size_t lcsa_sparse_attn_bwd_workspace_bytes(const lcsa_kv_cache* kv, int32_t q_frames);
+LCSA_API lcsa_status lcsa_sparse_attn_bwd(const lcsa_tensor* q, const lcsa_kv_cache* kv,
+                                 const int32_t* blk_idx, const int32_t* blk_cnt,
+                                 int32_t kmax, const lcsa_tensor* o, const float* lse,
+                                 const lcsa_tensor* d_o, lcsa_tensor* dq, void* dk, void* dv,
+                                 void* workspace, size_t workspace_bytes,
                                  lcsa_stream_t stream);
 
 /*
