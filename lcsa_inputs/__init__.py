@@ -185,6 +185,56 @@ def make_inputs(w: Workload):
     return {"q": torch.stack(qs), "k": ks, "v": vs, "workload": w}
 
 
+@dataclass(frozen=True)
+class SegmentWorkload:
+    """A batch of segments (video clips, or images as one-frame videos) for
+    dense attention confined to each segment; ``seg_frames[b]`` latent frames
+    in segment b, queries padded to the longest segment (padding frames are
+    the oldest positions and hold zeros)."""
+
+    name: str
+    H: int
+    D: int
+    Y: int
+    X: int
+    seg_frames: Tuple[int, ...]
+    seed: int = 0
+
+    @property
+    def B(self) -> int:
+        return len(self.seg_frames)
+
+    @property
+    def q_frames(self) -> int:
+        return max(self.seg_frames)
+
+    @property
+    def cap_frames(self) -> int:
+        return self.q_frames + (self.q_frames & 1)
+
+
+SEGMENT_WORKLOADS = {
+    # two 21-frame video clips (6 latent frames), one 13-frame clip (4) and one image
+    "joint": SegmentWorkload("joint", H=12, D=128, Y=48, X=88, seg_frames=(6, 6, 4, 1), seed=6),
+}
+
+
+def make_segment_inputs(w: SegmentWorkload):
+    """Draw Q, K, V of every segment (N(0,1), rounded to bf16). Returns
+    ``q`` bf16 ``[B][H][Tq][Y][X][D]`` (segment b in its newest seg_frames[b]
+    frames, zeros before) and per-segment lists ``k``, ``v`` of
+    ``[H][seg_frames[b]][Y][X][D]``."""
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    Tq = w.q_frames
+    q = torch.zeros((w.B, w.H, Tq, w.Y, w.X, w.D), dtype=torch.bfloat16)
+    ks, vs = [], []
+    for b, F in enumerate(w.seg_frames):
+        q[b, :, Tq - F:] = torch.randn((w.H, F, w.Y, w.X, w.D), generator=g).to(torch.bfloat16)
+        ks.append(torch.randn((w.H, F, w.Y, w.X, w.D), generator=g).to(torch.bfloat16))
+        vs.append(torch.randn((w.H, F, w.Y, w.X, w.D), generator=g).to(torch.bfloat16))
+    return {"q": q, "k": ks, "v": vs, "workload": w}
+
+
 def stacked(frames: List[torch.Tensor]) -> torch.Tensor:
     """Stack per-stream timelines of equal length into ``[B][H][F][Y][X][D]``."""
     return torch.stack(frames)

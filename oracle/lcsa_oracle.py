@@ -303,6 +303,28 @@ def attend_head_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, sel: Seque
 
 
 # --------------------------------------------------------------------------- #
+# 4c. Dense attention confined to one segment (section 2.2, stage 1: joint
+#     video-image training with a block-diagonal segment mask; an image is a
+#     one-frame video). Within a segment every query token sees every key
+#     token of the segment, past or future; nothing crosses segments.
+# --------------------------------------------------------------------------- #
+def segment_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """O [F_q][Y][X][D] and LSE [F_q][Y][X] of the segment's query tokens over
+    all of its key tokens (``attend_rows`` on the flattened tokens)."""
+    D = q.shape[-1]
+    o, lse = attend_rows(q.reshape(-1, D), k.reshape(-1, D), v.reshape(-1, D))
+    return o.reshape(q.shape), lse.reshape(q.shape[:3])
+
+
+def segment_attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, do: np.ndarray):
+    """dq, dk, dv of ``segment_attention`` (``attend_rows_backward`` on the
+    flattened tokens)."""
+    D = q.shape[-1]
+    dq, dk, dv = attend_rows_backward(q.reshape(-1, D), k.reshape(-1, D), v.reshape(-1, D), do.reshape(-1, D))
+    return dq.reshape(q.shape), dk.reshape(k.shape), dv.reshape(v.shape)
+
+
+# --------------------------------------------------------------------------- #
 # One (stream, head): pool -> scores -> masks -> top-K -> attention
 # --------------------------------------------------------------------------- #
 def select_head(qp: np.ndarray, kp: np.ndarray, q_frames: int, kv_frames: int, Y: int, X: int,

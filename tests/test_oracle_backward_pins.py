@@ -113,3 +113,46 @@ def test_gradient_closed_forms():
     v_eq = np.broadcast_to(v.reshape(-1, D)[0], v.reshape(-1, D).shape).reshape(v.shape).copy()
     dq0, dk0, _ = orc.attend_head_backward(q, k, v_eq, sel, g)
     assert np.abs(dq0).max() < 1e-12 and np.abs(dk0).max() < 1e-12
+
+
+def test_segment_attention_is_textbook_dense_attention():
+    """Within a segment: torch's scaled-dot-product attention (float64, no mask)."""
+    rng = np.random.default_rng(21)
+    q = rng.standard_normal((3, 8, 8, 16))
+    k = rng.standard_normal((3, 8, 8, 16))
+    v = rng.standard_normal((3, 8, 8, 16))
+    o, lse = orc.segment_attention(q, k, v)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q.reshape(1, -1, 16)), torch.tensor(k.reshape(1, -1, 16)), torch.tensor(v.reshape(1, -1, 16)))
+    np.testing.assert_allclose(o.reshape(-1, 16), ref[0].numpy(), rtol=1e-12, atol=1e-12)
+    s = (q.reshape(-1, 16) @ k.reshape(-1, 16).T) / 4.0
+    np.testing.assert_allclose(lse.reshape(-1), np.log(np.exp(s).sum(axis=1)), rtol=1e-12)
+
+
+def test_segments_equal_block_diagonal_mask_on_a_packed_sequence():
+    """Two segments packed into one sequence with a block-diagonal boolean mask
+    (torch autograd, float64) give each segment's own attention and gradients."""
+    rng = np.random.default_rng(23)
+    F = (2, 1)   # a two-frame clip and an image
+    segs = [(rng.standard_normal((f, 8, 8, 16)), rng.standard_normal((f, 8, 8, 16)),
+             rng.standard_normal((f, 8, 8, 16)), rng.standard_normal((f, 8, 8, 16))) for f in F]
+    n = [f * 64 for f in F]
+    mask = torch.zeros((sum(n), sum(n)), dtype=torch.bool)
+    mask[:n[0], :n[0]] = True
+    mask[n[0]:, n[0]:] = True
+    tq = torch.tensor(np.concatenate([s[0].reshape(-1, 16) for s in segs]), requires_grad=True)
+    tk = torch.tensor(np.concatenate([s[1].reshape(-1, 16) for s in segs]), requires_grad=True)
+    tv = torch.tensor(np.concatenate([s[2].reshape(-1, 16) for s in segs]), requires_grad=True)
+    g = torch.tensor(np.concatenate([s[3].reshape(-1, 16) for s in segs]))
+    sc = (tq @ tk.T / 4.0).masked_fill(~mask, float("-inf"))
+    o = torch.softmax(sc, dim=1) @ tv
+    (o * g).sum().backward()
+    off = 0
+    for (q, k, v, do), m in zip(segs, n):
+        ro, _ = orc.segment_attention(q, k, v)
+        dq, dk, dv = orc.segment_attention_backward(q, k, v, do)
+        np.testing.assert_allclose(ro.reshape(-1, 16), o[off:off + m].detach().numpy(), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dq.reshape(-1, 16), tq.grad[off:off + m].numpy(), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dk.reshape(-1, 16), tk.grad[off:off + m].numpy(), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dv.reshape(-1, 16), tv.grad[off:off + m].numpy(), rtol=1e-10, atol=1e-12)
+        off += m
