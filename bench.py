@@ -528,6 +528,87 @@ def run_backward(args, world, rank, local):
     return line
 
 
+def run_segment(args, world, rank, local):
+    """Stage-1 dense attention confined to segments (video clips and images):
+    segment block lists, then the attention forward and backward; each step is
+    one forward and one backward of the batch (the block lists are built once)."""
+    import block_sparse_causal_lcsa_b200 as lc
+
+    w = li.SEGMENT_WORKLOADS["joint"]
+    w = li.SegmentWorkload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    x = li.make_segment_inputs(w)
+    cache = lc.KVCache(w.B, w.H, w.cap_frames, w.Y, w.X, w.D, device=dev)
+    for b in range(w.B):
+        lc.kv_append(cache, x["k"][b].unsqueeze(0).to(dev), x["v"][b].unsqueeze(0).to(dev), stream_offset=b)
+    q = x["q"].to(dev)
+    idx, cnt = lc.segment_blocks(w.q_frames, cache)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:5], dtype=torch.float32, device=dev)
+    g = torch.Generator().manual_seed(w.seed + 11)
+    d_o = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    for b, F in enumerate(w.seg_frames):
+        d_o[b, :, :w.q_frames - F] = 0
+    d_o = d_o.to(dev)
+    dq, dk, dv = torch.empty_like(q), torch.zeros_like(cache.k), torch.zeros_like(cache.v)
+    ws = torch.empty(max(lc.sparse_attn_bwd_workspace_bytes(cache, w.q_frames), 16), dtype=torch.uint8, device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record()
+        lc.sparse_attn_fwd(q, cache, idx, cnt, o, lse)
+        if ev is not None:
+            ev[1].record()
+        lc.sparse_attn_bwd(q, cache, idx, cnt, o, lse, d_o, dq, dk, dv, ws)
+        if ev is not None:
+            ev[2].record()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if lc.last_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for ev in evs:
+        flush.zero_()
+        step(ev)
+    torch.cuda.synchronize()
+    barrier(world)
+    time.sleep(0.2)
+    clk = clocks.stop()
+    if lc.last_device_error() != 0:
+        raise RuntimeError("device error during the timed steps")
+    fwd_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in evs), world)
+    bwd_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in evs), world)
+    fwd_flops = attn_flops(cnt, idx, cache, w.Y // 8, w.X // 8, w.D)
+    f_tf = fwd_flops / (fwd_ms / 1e3) / 1e12
+    b_tf = 2.5 * fwd_flops / (bwd_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
+    return {
+        "metric": "ms per attention forward + backward of a stage-1 joint batch (block-diagonal segment mask)",
+        "value": round((fwd_ms + bwd_ms) / world, 4), "unit": "ms/batch", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(fwd_ms + bwd_ms, 4), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1))",
+        "config": {"workload": "768x1408 joint batch: segments of %s latent frames (images are one frame), "
+                               "12 heads, d=128, dense within each segment" % (w.seg_frames,),
+                   "name": "joint", "mode": "segment", "l2": "flushed before every timed step (512 MB write)"},
+        "per_kernel_ms": {"attn_fwd": round(fwd_ms, 4), "attn_bwd": round(bwd_ms, 4)},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd", "achieved": round(f_tf, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(f_tf / peak, 4), "flops_per_launch": fwd_flops, "traffic": None,
+                     "bwd_achieved": round(b_tf, 2), "bwd_frac": round(b_tf / peak, 4)},
+        "gpu_launches": 5 * args.steps,
+        "clocks": clk,
+    }
+
+
 def _threads():
     try:
         from threadpoolctl import threadpool_info
@@ -599,8 +680,9 @@ def main():
     ap.add_argument("--workload", default="chunk", choices=sorted(WORKLOAD_TEXT))
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="fwd", choices=["fwd", "bwd"],
-                    help="fwd: the streaming step (default); bwd: the attention backward on a clip")
+    ap.add_argument("--mode", default="fwd", choices=["fwd", "bwd", "segment"],
+                    help="fwd: the streaming step (default); bwd: the attention backward on a clip; "
+                         "segment: stage-1 dense segment attention, forward + backward")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -617,6 +699,8 @@ def main():
             if args.workload == "chunk":
                 args.workload = "clip"
             line = run_backward(args, world, rank, local)
+        elif args.mode == "segment":
+            line = run_segment(args, world, rank, local)
         else:
             line = run_ours(args, world, rank, local)
         if rank == 0:

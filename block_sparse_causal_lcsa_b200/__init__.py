@@ -18,6 +18,7 @@ from .api import (  # noqa: F401
     kv_append,
     last_device_error,
     pool_qk,
+    segment_blocks,
     select_blocks,
     select_blocks_noalloc,
     select_kmax,

@@ -76,6 +76,9 @@ PROTOTYPES = {
     "lcsa_sparse_attn_fwd": (C.c_int, [C.POINTER(Tensor), C.POINTER(KVCacheStruct), C.c_void_p,
                                        C.c_void_p, C.c_int32, C.POINTER(Tensor), C.c_void_p,
                                        C.c_void_p]),
+    "lcsa_segment_kmax": (C.c_int32, [C.POINTER(KVCacheStruct)]),
+    "lcsa_segment_blocks": (C.c_int, [C.c_int32, C.POINTER(KVCacheStruct), C.c_int32, C.c_void_p, C.c_void_p,
+                                      C.c_void_p]),
     "lcsa_sparse_attn_bwd_workspace_bytes": (C.c_size_t, [C.POINTER(KVCacheStruct), C.c_int32]),
     "lcsa_sparse_attn_bwd": (C.c_int, [C.POINTER(Tensor), C.POINTER(KVCacheStruct), C.c_void_p, C.c_void_p,
                                        C.c_int32, C.POINTER(Tensor), C.c_void_p, C.POINTER(Tensor),

@@ -232,6 +232,24 @@ def sparse_attn_fwd(q: torch.Tensor, cache: KVCache, blk_idx: torch.Tensor, blk_
     return o, lse
 
 
+def segment_blocks(q_frames: int, cache: KVCache, kmax: Optional[int] = None,
+                   blk_idx: Optional[torch.Tensor] = None, blk_cnt: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None):
+    """Block lists for dense attention inside each stream (segment) of the cache:
+    (blk_idx [B,H,nQB,kmax], blk_cnt [B,H,nQB]) for sparse_attn_fwd / _bwd."""
+    if kmax is None:
+        kmax = int(_lib.lcsa_segment_kmax(C.byref(cache.struct)))
+    nQB = ((q_frames + 1) // 2) * (cache.Y // 8) * (cache.X // 8)
+    dev = cache.k.device
+    if blk_idx is None:
+        blk_idx = torch.empty((cache.B, cache.H, nQB, kmax), dtype=torch.int32, device=dev)
+    if blk_cnt is None:
+        blk_cnt = torch.empty((cache.B, cache.H, nQB), dtype=torch.int32, device=dev)
+    _check(_lib.lcsa_segment_blocks(q_frames, C.byref(cache.struct), blk_idx.shape[-1], blk_idx.data_ptr(),
+                                    blk_cnt.data_ptr(), _stream(stream)), "lcsa_segment_blocks")
+    return blk_idx, blk_cnt
+
+
 def sparse_attn_bwd_workspace_bytes(cache: KVCache, q_frames: int) -> int:
     return int(_lib.lcsa_sparse_attn_bwd_workspace_bytes(C.byref(cache.struct), q_frames))
 

@@ -15,6 +15,7 @@
 #include "attn_bwd.cuh"
 #include "kv_append.cuh"
 #include "ingest.cuh"
+#include "segment.cuh"
 #include "select.cuh"
 
 // Scratch of lcsa_select_blocks_noalloc: the score keys that the caller's
@@ -444,6 +445,46 @@ lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames, const lcs
   return launched();
 }
 
+int32_t lcsa_segment_kmax(const lcsa_kv_cache* kv) {
+  if (kv == nullptr || kv->B < 1 || kv->B > LCSA_MAX_STREAMS || kv->Y < 8 || kv->X < 8) return 0;
+  int nKT = 0;
+  for (int b = 0; b < kv->B; ++b) {
+    const int n = static_cast<int>((kv->end[b] >> 1) - (kv->begin[b] >> 1));
+    nKT = n > nKT ? n : nKT;
+  }
+  return nKT * (kv->Y / 8) * (kv->X / 8);
+}
+
+lcsa_status lcsa_segment_blocks(int32_t q_frames, const lcsa_kv_cache* kv, int32_t kmax, int32_t* blk_idx,
+                                int32_t* blk_cnt, lcsa_stream_t stream) {
+  lcsa_status s = check_cache(kv);
+  if (s != LCSA_OK) return s;
+  if (blk_idx == nullptr || blk_cnt == nullptr) return LCSA_ERR_INVALID_ARG;
+  if (q_frames < 1) return LCSA_ERR_SHAPE;
+  for (int b = 0; b < kv->B; ++b)
+    if (kv->end[b] - kv->begin[b] < 1 || kv->end[b] - kv->begin[b] > q_frames) return LCSA_ERR_SHAPE;
+  if (kmax < lcsa_segment_kmax(kv)) return LCSA_ERR_CAPACITY;
+  const int64_t rows = static_cast<int64_t>(kv->B) * kv->H * temporal_blocks(q_frames) * (kv->Y / 8) * (kv->X / 8);
+  if (rows * 32 > 0x7fffffff) return LCSA_ERR_SHAPE;
+  int dev;
+  unsigned int* err;
+  if ((s = device_setup(&dev, &err)) != LCSA_OK) return s;
+  SegmentParams p{};
+  p.blk_idx = blk_idx;
+  p.blk_cnt = blk_cnt;
+  p.H = kv->H;
+  p.Tq = q_frames;
+  p.nQT = temporal_blocks(q_frames);
+  p.HbWb = (kv->Y / 8) * (kv->X / 8);
+  p.kmax = kmax;
+  p.rows = rows;
+  for (int b = 0; b < kv->B; ++b) { p.kv_begin[b] = kv->begin[b]; p.kv_end[b] = kv->end[b]; }
+  // one warp per query-block row, rows numbered bh * nQB + qb
+  segment_blocks_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0,
+                          static_cast<cudaStream_t>(stream)>>>(p);
+  return launched();
+}
+
 // Backward workspace: LSE*log2(e) and delta per query row in block order,
 // then the per-key-block count and list of the query blocks that kept it.
 struct BwdSizes {
@@ -493,7 +534,7 @@ lcsa_status lcsa_sparse_attn_bwd(const lcsa_tensor* q, const lcsa_kv_cache* kv, 
     if (t->B != q->B || t->H != q->H || t->T != q->T || t->Y != q->Y || t->X != q->X || t->D != q->D)
       return LCSA_ERR_SHAPE;
   for (int b = 0; b < kv->B; ++b)
-    if (kv->end[b] - kv->begin[b] < q->T) return LCSA_ERR_SHAPE;
+    if (kv->end[b] - kv->begin[b] < 1) return LCSA_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(lse) & 3u) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
     return LCSA_ERR_ALIGN;
   const BwdSizes z = bwd_sizes(kv, q->T);
@@ -608,7 +649,7 @@ lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_cache* kv, 
   if (o->B != q->B || o->H != q->H || o->T != q->T || o->Y != q->Y || o->X != q->X || o->D != q->D)
     return LCSA_ERR_SHAPE;
   for (int b = 0; b < kv->B; ++b)
-    if (kv->end[b] - kv->begin[b] < q->T) return LCSA_ERR_SHAPE;
+    if (kv->end[b] - kv->begin[b] < 1) return LCSA_ERR_SHAPE;
   if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LCSA_ERR_ALIGN;
   int dev;
   unsigned int* err;

@@ -271,7 +271,8 @@ LCSA_API lcsa_status lcsa_select_blocks_noalloc(const double* q_pool, int32_t q_
  * stage 2: "apply full attention within the selected regions").
  *
  * q        token tensor [B][H][Tq][Y][X][D]: the newest Tq frames of each
- *          stream of kv.
+ *          stream of kv (a stream holding fewer frames has padding query
+ *          frames, see lcsa_segment_blocks).
  * kv       cache holding K and V (B, H, Y, X, D as q).
  * blk_idx, blk_cnt, kmax  as written by lcsa_select_blocks (device).
  * o        token tensor like q (bf16), device; receives
@@ -286,6 +287,27 @@ LCSA_API lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_ca
                                  const int32_t* blk_idx, const int32_t* blk_cnt,
                                  int32_t kmax, lcsa_tensor* o, float* lse,
                                  lcsa_stream_t stream);
+
+/*
+ * lcsa_segment_blocks - block lists for dense attention confined to one
+ * segment (section 2.2, stage 1: joint video-image training with a
+ * block-diagonal segment mask, so that attention stays inside one video clip
+ * or one image; an image is a one-frame video).
+ *
+ * Each stream of kv is one segment: its cached frames [begin, end), 1 to
+ * q_frames of them. The query tensor of the attention calls has q_frames
+ * frames per stream; segment b's queries are its newest end-begin frames and
+ * older query frames are padding. Every query block holding at least one of
+ * the segment's frames keeps every key block of the segment, ascending (no
+ * causal limit, no top-K); a query block of padding only keeps none, so the
+ * forward writes zeros and LSE = -inf there (pass dO = 0 for padding rows to
+ * the backward). blk_idx [B][H][nQB][kmax], blk_cnt [B][H][nQB] as for
+ * lcsa_select_blocks; kmax >= lcsa_segment_kmax(kv), else LCSA_ERR_CAPACITY.
+ * The lists feed lcsa_sparse_attn_fwd / lcsa_sparse_attn_bwd unchanged.
+ */
+LCSA_API int32_t lcsa_segment_kmax(const lcsa_kv_cache* kv);
+LCSA_API lcsa_status lcsa_segment_blocks(int32_t q_frames, const lcsa_kv_cache* kv, int32_t kmax,
+                                int32_t* blk_idx, int32_t* blk_cnt, lcsa_stream_t stream);
 
 /*
  * lcsa_sparse_attn_bwd - gradients of lcsa_sparse_attn_fwd for training with
