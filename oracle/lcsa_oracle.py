@@ -44,6 +44,8 @@ import numpy as np
 
 BLOCK_T, BLOCK_Y, BLOCK_X = 2, 8, 8
 WINDOW_TRUNCATE, WINDOW_PRESERVE = 0, 1
+WINDOW_TRUNCATE_TOKENS = 2   # token-level window, clipped at the frame edge
+WINDOW_PRESERVE_TOKENS = 3   # token-level window, shifted inward at the edge
 TIE_EPS = 1e-5
 
 # Largest exponent spread (in binades) among the non-zero terms of one block sum
@@ -157,6 +159,33 @@ def window_range(i: int, n: int, window: int, mode: int) -> Tuple[int, int]:
     raise ValueError("unknown window mode")
 
 
+def token_window_range(p: int, n: int, window: int, mode: int) -> Tuple[int, int]:
+    """Half-open range of token coordinates along one axis seen from query token p.
+
+    Token-level reading of "each query's attention is limited to a local
+    neighbourhood" (e.g. 1152 px = 72 tokens): the window is ``window`` tokens
+    wide with the query at offset window // 2 (window // 2 tokens before it,
+    the rest after), truncated at the frame edge or, with preserve, shifted
+    inward so it keeps its width (start = max(0, min(p - window//2, n - window))).
+    """
+    s = p - window // 2
+    if mode == WINDOW_TRUNCATE_TOKENS:
+        return max(0, s), min(n, s + window)
+    if mode == WINDOW_PRESERVE_TOKENS:
+        st = max(0, min(s, n - window))
+        return st, min(n, st + window)
+    raise ValueError("unknown token window mode")
+
+
+def token_block_range(i: int, n_tokens: int, window: int, mode: int) -> Tuple[int, int]:
+    """Half-open range of block coordinates along one axis holding at least one
+    token that some token of block i sees (the union of its tokens' windows;
+    both window ends move monotonically with the query token)."""
+    lo = token_window_range(BLOCK_Y * i, n_tokens, window, mode)[0]
+    hi = token_window_range(BLOCK_Y * i + BLOCK_Y - 1, n_tokens, window, mode)[1]
+    return lo // BLOCK_Y, (hi - 1) // BLOCK_Y + 1
+
+
 def allowed_blocks(tq: int, yq: int, xq: int, nKT: int, Hb: int, Wb: int,
                    window: int = 0, mode: int = WINDOW_TRUNCATE) -> np.ndarray:
     """Boolean mask over the nKT*Hb*Wb key blocks for query block (tq, yq, xq).
@@ -167,6 +196,11 @@ def allowed_blocks(tq: int, yq: int, xq: int, nKT: int, Hb: int, Wb: int,
     applies at every past time step.
     """
     m = np.zeros((nKT, Hb, Wb), dtype=bool)
+    if window > 0 and mode in (WINDOW_TRUNCATE_TOKENS, WINDOW_PRESERVE_TOKENS):
+        y0, y1 = token_block_range(yq, Hb * BLOCK_Y, window, mode)
+        x0, x1 = token_block_range(xq, Wb * BLOCK_X, window, mode)
+        m[:tq + 1, y0:y1, x0:x1] = True
+        return m.reshape(-1)
     y0, y1 = (0, Hb) if window <= 0 else window_range(yq, Hb, window, mode)
     x0, x1 = (0, Wb) if window <= 0 else window_range(xq, Wb, window, mode)
     m[:tq + 1, y0:y1, x0:x1] = True
@@ -222,6 +256,31 @@ def attend_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> Tuple[np.ndarray
     e = np.exp(s - mx)
     l = e.sum(axis=1, keepdims=True)
     return (e / l) @ v, mx[:, 0] + np.log(l[:, 0])
+
+
+def attend_rows_masked(q: np.ndarray, k: np.ndarray, v: np.ndarray,
+                       mask: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """``attend_rows`` with a boolean visibility mask [n][m]: masked keys get
+    zero weight. A row that sees no key at all has O = 0 and LSE = -inf."""
+    s = (q @ k.T) / math.sqrt(q.shape[1])
+    s = np.where(mask, s, -np.inf)
+    mx = s.max(axis=1, keepdims=True)
+    empty = ~np.isfinite(mx[:, 0])
+    mx = np.where(np.isfinite(mx), mx, 0.0)
+    e = np.where(mask, np.exp(s - mx), 0.0)
+    l = e.sum(axis=1, keepdims=True)
+    o = (e / np.where(l > 0, l, 1.0)) @ v
+    lse = mx[:, 0] + np.log(np.where(l[:, 0] > 0, l[:, 0], 1.0))
+    o[empty] = 0.0
+    lse[empty] = -np.inf
+    return o, lse
+
+
+def token_yx(F: int, Y: int, X: int, ids: Sequence[int]) -> Tuple[np.ndarray, np.ndarray]:
+    """(y, x) token coordinates of the tokens of the given blocks, in the order
+    ``gather_blocks`` concatenates them."""
+    flat = block_token_index(F, Y, X, ids) % (Y * X)
+    return flat // X, flat % X
 
 
 def gather_blocks(x: np.ndarray, ids: Sequence[int]) -> np.ndarray:
@@ -355,7 +414,7 @@ def select_head(qp: np.ndarray, kp: np.ndarray, q_frames: int, kv_frames: int, Y
 
 
 def attend_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, sel: Sequence[np.ndarray],
-                rows: Sequence[int] | None = None):
+                rows: Sequence[int] | None = None, window: int = 0, mode: int = WINDOW_TRUNCATE):
     """Attention output of one (stream, head) for the given selections.
 
     ``q`` [Tq][Y][X][D], ``k``/``v`` [F][Y][X][D] float64. Returns O laid out
@@ -371,7 +430,19 @@ def attend_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, sel: Sequence[np.nd
         t, r = divmod(int(i), Hb * Wb)
         yb, xb = divmod(r, Wb)
         qi = block_token_view(q, qtb[t], yb, xb)
-        o, lse = attend_rows(qi, gather_blocks(k, sel[i]), gather_blocks(v, sel[i]))
+        if window > 0 and mode in (WINDOW_TRUNCATE_TOKENS, WINDOW_PRESERVE_TOKENS):
+            # token-level window inside the kept blocks: key (yk, xk) is visible
+            # to query (yq, xq) iff yk and xk lie in the query token's windows
+            qy, qx = token_yx(Tq, Y, X, [i])
+            ky, kx = token_yx(k.shape[0], Y, X, sel[i])
+            vis = np.ones((qy.size, ky.size), dtype=bool)
+            for a, (yy, xx) in enumerate(zip(qy, qx)):
+                y0, y1 = token_window_range(int(yy), Y, window, mode)
+                x0, x1 = token_window_range(int(xx), X, window, mode)
+                vis[a] = (ky >= y0) & (ky < y1) & (kx >= x0) & (kx < x1)
+            o, lse = attend_rows_masked(qi, gather_blocks(k, sel[i]), gather_blocks(v, sel[i]), vis)
+        else:
+            o, lse = attend_rows(qi, gather_blocks(k, sel[i]), gather_blocks(v, sel[i]))
         ys, xs = slice(yb * BLOCK_Y, (yb + 1) * BLOCK_Y), slice(xb * BLOCK_X, (xb + 1) * BLOCK_X)
         O[qtb[t], ys, xs, :] = o.reshape(len(qtb[t]), BLOCK_Y, BLOCK_X, D)
         L[qtb[t], ys, xs] = lse.reshape(len(qtb[t]), BLOCK_Y, BLOCK_X)
@@ -385,7 +456,7 @@ def lcsa_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, top_k: int = 0,
     qp, kp = pool_blocks(q), pool_blocks(k)
     sel, Ks, Cs = select_head(qp, kp, q.shape[0], k.shape[0], q.shape[1], q.shape[2],
                               top_k, density, window, mode, eps)
-    O, L = attend_head(q, k, v, sel, rows)
+    O, L = attend_head(q, k, v, sel, rows, window, mode)
     return {"q_pool": qp, "k_pool": kp, "sel": sel, "K": Ks, "C": Cs, "O": O, "LSE": L}
 
 
