@@ -41,6 +41,10 @@ WORKLOAD_TEXT = {
     "multistream": "4 streams at 768x1408, 2-frame chunks, ragged 4/5/6 past frames, 13.6%",
     "uhr_truncate": "1536x2688: 96x168 tokens/frame, 2+4 frames, 9x9-block window, truncate, 13.6%",
     "uhr_preserve": "1536x2688: 96x168 tokens/frame, 2+4 frames, 9x9-block window, preserve, 13.6%",
+    "uhr_truncate_tok": "1536x2688: 96x168 tokens/frame, 2+4 frames, 72x72-token window per query token, "
+                        "truncate, 13.6%",
+    "uhr_preserve_tok": "1536x2688: 96x168 tokens/frame, 2+4 frames, 72x72-token window per query token, "
+                        "preserve, 13.6%",
     "clip": "whole 101-frame clip at 768x1408: 26 latent frames, block-causal, 13.6%",
     "clip_5": "whole 101-frame clip at 768x1408: 26 latent frames, block-causal, 5%",
     "clip_30": "whole 101-frame clip at 768x1408: 26 latent frames, block-causal, 30%",

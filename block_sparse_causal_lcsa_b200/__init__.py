@@ -11,7 +11,9 @@ from .api import (  # noqa: F401
     SelectParams,
     StreamingStep,
     WINDOW_PRESERVE,
+    WINDOW_PRESERVE_TOKENS,
     WINDOW_TRUNCATE,
+    WINDOW_TRUNCATE_TOKENS,
     debug_exp2_poly,
     debug_set_wait_limit_ns,
     debug_stalled_wait,

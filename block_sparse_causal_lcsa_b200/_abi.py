@@ -23,6 +23,8 @@ ERR_CUDA = -6
 ERR_TIMEOUT = -7
 ERR_DEVICE_BOUNDS = -8
 ERR_SCRATCH_LIMIT = -9
+WINDOW_TRUNCATE_TOKENS = 2
+WINDOW_PRESERVE_TOKENS = 3
 SELECT_STATIC_SCRATCH_BYTES = 8 << 20
 
 WINDOW_TRUNCATE = 0
@@ -76,6 +78,9 @@ PROTOTYPES = {
     "lcsa_sparse_attn_fwd": (C.c_int, [C.POINTER(Tensor), C.POINTER(KVCacheStruct), C.c_void_p,
                                        C.c_void_p, C.c_int32, C.POINTER(Tensor), C.c_void_p,
                                        C.c_void_p]),
+    "lcsa_sparse_attn_fwd_window": (C.c_int, [C.POINTER(Tensor), C.POINTER(KVCacheStruct), C.c_void_p, C.c_void_p,
+                                              C.c_int32, C.c_int32, C.c_int32, C.POINTER(Tensor), C.c_void_p,
+                                              C.c_void_p]),
     "lcsa_segment_kmax": (C.c_int32, [C.POINTER(KVCacheStruct)]),
     "lcsa_segment_blocks": (C.c_int, [C.c_int32, C.POINTER(KVCacheStruct), C.c_int32, C.c_void_p, C.c_void_p,
                                       C.c_void_p]),

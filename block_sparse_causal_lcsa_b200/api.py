@@ -22,6 +22,8 @@ _lib = _abi.load()
 OK = _abi.OK
 WINDOW_TRUNCATE = _abi.WINDOW_TRUNCATE
 WINDOW_PRESERVE = _abi.WINDOW_PRESERVE
+WINDOW_TRUNCATE_TOKENS = _abi.WINDOW_TRUNCATE_TOKENS
+WINDOW_PRESERVE_TOKENS = _abi.WINDOW_PRESERVE_TOKENS
 TIE_EPS = 1e-5
 
 
@@ -216,8 +218,11 @@ def select_blocks_noalloc(q_pool: torch.Tensor, q_frames: int, cache: KVCache, p
 
 def sparse_attn_fwd(q: torch.Tensor, cache: KVCache, blk_idx: torch.Tensor, blk_cnt: torch.Tensor,
                     o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                    with_lse: bool = True, stream: Optional[torch.cuda.Stream] = None):
-    """Attention of the query chunk over its kept key blocks: (O bf16 like q, LSE fp32)."""
+                    with_lse: bool = True, stream: Optional[torch.cuda.Stream] = None,
+                    window: int = 0, window_mode: int = WINDOW_TRUNCATE_TOKENS):
+    """Attention of the query chunk over its kept key blocks: (O bf16 like q, LSE fp32).
+    With ``window`` > 0 (a token-level window mode), each query token only sees
+    the key tokens inside its window (lcsa_sparse_attn_fwd_window)."""
     if o is None:
         o = torch.empty_like(q)
     if lse is None and with_lse:
@@ -225,10 +230,17 @@ def sparse_attn_fwd(q: torch.Tensor, cache: KVCache, blk_idx: torch.Tensor, blk_
     if not blk_idx.is_contiguous() or not blk_cnt.is_contiguous():
         raise ValueError("blk_idx and blk_cnt must be contiguous")
     qd, od = tensor_desc(q), tensor_desc(o)
-    _check(_lib.lcsa_sparse_attn_fwd(C.byref(qd), C.byref(cache.struct), blk_idx.data_ptr(),
-                                     blk_cnt.data_ptr(), blk_idx.shape[-1], C.byref(od),
-                                     lse.data_ptr() if lse is not None else None, _stream(stream)),
-           "lcsa_sparse_attn_fwd")
+    lse_ptr = lse.data_ptr() if lse is not None else None
+    if window > 0:
+        _check(_lib.lcsa_sparse_attn_fwd_window(C.byref(qd), C.byref(cache.struct), blk_idx.data_ptr(),
+                                                blk_cnt.data_ptr(), blk_idx.shape[-1], window, window_mode,
+                                                C.byref(od), lse_ptr, _stream(stream)),
+               "lcsa_sparse_attn_fwd_window")
+    else:
+        _check(_lib.lcsa_sparse_attn_fwd(C.byref(qd), C.byref(cache.struct), blk_idx.data_ptr(),
+                                         blk_cnt.data_ptr(), blk_idx.shape[-1], C.byref(od), lse_ptr,
+                                         _stream(stream)),
+               "lcsa_sparse_attn_fwd")
     return o, lse
 
 
@@ -342,5 +354,7 @@ class StreamingStep:
         kv_append(self.cache, k_new, v_new, None, 0, stream)
         select_blocks(self.q_pool, self.q_frames, self.cache, self.params, self.kmax,
                       self.blk_idx, self.blk_cnt, self.workspace, stream)
-        sparse_attn_fwd(q, self.cache, self.blk_idx, self.blk_cnt, self.o, self.lse, stream=stream)
+        tw = self.params.window if self.params.window_mode >= WINDOW_TRUNCATE_TOKENS else 0
+        sparse_attn_fwd(q, self.cache, self.blk_idx, self.blk_cnt, self.o, self.lse, stream=stream,
+                        window=tw, window_mode=self.params.window_mode)
         return self.o, self.lse

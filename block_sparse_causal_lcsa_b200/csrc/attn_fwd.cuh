@@ -86,6 +86,7 @@ struct AttnParams {
   float* lse;                // [B*H][Tq][Y][X] or null
   int64_t osh, ost, osy, osx;  // strides of o (stream stride = H * osh)
   int32_t H, Tq, Y, X, Hb, Wb, nQT, nQB, kmax, cap;
+  int32_t win, win_mode;     // token-level window (0: none), mode 2 truncate / 3 preserve
   float scale_log2;          // log2(e) / sqrt(D)
   uint64_t wait_limit_ns;
   unsigned int* err;
@@ -320,9 +321,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     float m_run = -INFINITY, l_run = 0.f;         // running max (log2 units) and sum
     bool done = n > 0;
     int next_blk = n > 0 ? checked(blist[0]) : 0;
+    // token-level window of this row's query token (a key token is visible iff
+    // its y and x lie in these ranges)
+    int wy0 = 0, wy1 = 0, wx0 = 0, wx1 = 0;
+    if (p.win > 0) {
+      token_window(8 * yq + ((r >> 3) & 7), p.Y, p.win, p.win_mode, wy0, wy1);
+      token_window(8 * xq + (r & 7), p.X, p.win, p.win_mode, wx0, wx1);
+    }
     for (int j = 0; j < n; ++j) {
       const int sb = j % S_BUFS;
-      const bool partial = oldest_partial && next_blk < HbWb;
+      const int blk = next_blk;
+      const bool partial = oldest_partial && blk < HbWb;
       if (j + 1 < n) next_blk = checked(blist[j + 1]);
       if (!warp_wait(bar(B_S_FULL + sb), (j / S_BUFS) & 1, w)) { done = false; break; }
       tc_fence_after();
@@ -335,6 +344,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (partial) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = __float_as_uint(-INFINITY);
+      }
+      if (p.win > 0) {
+        // rows / columns of the key block (8 x 8 tokens, both frames alike) inside the window
+        const int spk = blk % HbWb;
+        const int ry = 8 * (spk / p.Wb), rx = 8 * (spk % p.Wb);
+        const int ylo = min(max(wy0 - ry, 0), 8), yhi = min(max(wy1 - ry, 0), 8);
+        const int xlo = min(max(wx0 - rx, 0), 8), xhi = min(max(wx1 - rx, 0), 8);
+        const uint32_t ym = ((1u << yhi) - 1u) & ~((1u << ylo) - 1u);
+        const uint32_t xm = ((1u << xhi) - 1u) & ~((1u << xlo) - 1u);
+        if (ym != 0xFFu || xm != 0xFFu) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (!((ym >> ((c >> 3) & 7)) & (xm >> (c & 7)) & 1u)) s[c] = __float_as_uint(-INFINITY);
+        }
       }
       float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
@@ -351,7 +374,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // O may only be rescaled once PV_{j-1} has finished
         if (!warp_wait(bar(B_PV_DONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, w)) { done = false; break; }
         tc_fence_after();
-        const float alpha = ex2_approx(m_run - m_new);
+        // 1 for rows whose max did not change (also rows still at -inf, where the difference is NaN)
+        const float alpha = m_new == m_run ? 1.f : ex2_approx(m_run - m_new);
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
@@ -365,7 +389,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         l_run *= alpha;
       }
       m_run = m_new;
-      const uint64_t nm2 = f2_pack(-m_run, -m_run);
+      // a row that has seen no visible key yet keeps m = -inf; its exponentials use 0
+      const float m_ref = m_run == -INFINITY ? 0.f : m_run;
+      const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
       uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = f2_pack(0.f, 0.f);
       uint32_t pk[64];
 #pragma unroll
@@ -407,7 +433,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                           static_cast<int64_t>(y) * p.osy + static_cast<int64_t>(x) * p.osx;
     if (done) {
       tc_fence_after();
-      const float inv_l = 1.f / l_run;
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;   // a row with no visible key: O = 0
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
@@ -425,7 +451,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       if (p.lse != nullptr && row_valid)
         p.lse[((static_cast<int64_t>(bh) * p.Tq + frame) * p.Y + y) * p.X + x] =
-            (m_run + log2f(l_run)) * 0.69314718055994531f;
+            l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     } else if (n == 0 && row_valid) {
       // no kept block (cannot happen for selections made by this library)
       uint4* dst = reinterpret_cast<uint4*>(orow);

@@ -176,8 +176,19 @@ int32_t kmax_for(int nKT, int nQT, int Hb, int Wb, const lcsa_select_params* p) 
   if (nKT < nQT || nQT < 1) return 0;
   int wy = Hb, wx = Wb;
   if (p->window > 0) {
-    wy = p->window < Hb ? p->window : Hb;
-    wx = p->window < Wb ? p->window : Wb;
+    // widest window over all query blocks along each axis
+    wy = 0;
+    wx = 0;
+    for (int i = 0; i < Hb; ++i) {
+      int lo, hi;
+      window_bounds(i, Hb, p->window, p->window_mode, lo, hi);
+      wy = hi - lo > wy ? hi - lo : wy;
+    }
+    for (int i = 0; i < Wb; ++i) {
+      int lo, hi;
+      window_bounds(i, Wb, p->window, p->window_mode, lo, hi);
+      wx = hi - lo > wx ? hi - lo : wx;
+    }
   }
   const int C = nKT * wy * wx;
   if (p->top_k > 0) return p->top_k < C ? p->top_k : C;
@@ -393,8 +404,10 @@ lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames, const lcs
   if (!aligned16(q_pool) || !aligned16(workspace)) return LCSA_ERR_ALIGN;
   if (sp->top_k < 0 || sp->kmax < 1 || !(sp->tie_eps >= 0.0)) return LCSA_ERR_INVALID_ARG;
   if (sp->top_k == 0 && !(sp->density > 0.0 && sp->density <= 1.0)) return LCSA_ERR_INVALID_ARG;
-  if (sp->window < 0 || (sp->window > 0 && sp->window % 2 == 0)) return LCSA_ERR_INVALID_ARG;
-  if (sp->window_mode != LCSA_WINDOW_TRUNCATE && sp->window_mode != LCSA_WINDOW_PRESERVE)
+  if (sp->window_mode < LCSA_WINDOW_TRUNCATE || sp->window_mode > LCSA_WINDOW_PRESERVE_TOKENS)
+    return LCSA_ERR_INVALID_ARG;
+  // block windows are centred: an odd number of blocks; token windows any width
+  if (sp->window < 0 || (sp->window > 0 && sp->window % 2 == 0 && sp->window_mode <= LCSA_WINDOW_PRESERVE))
     return LCSA_ERR_INVALID_ARG;
   if (q_frames < 1) return LCSA_ERR_SHAPE;
   const int Hb = kv->Y / 8, Wb = kv->X / 8, HbWb = Hb * Wb;
@@ -635,9 +648,9 @@ lcsa_status lcsa_select_blocks_noalloc(const double* q_pool, int32_t q_frames, c
                             LCSA_SELECT_STATIC_SCRATCH_BYTES, stream);
 }
 
-lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_cache* kv, const int32_t* blk_idx,
-                                 const int32_t* blk_cnt, int32_t kmax, lcsa_tensor* o, float* lse,
-                                 lcsa_stream_t stream) {
+static lcsa_status attn_fwd_impl(const lcsa_tensor* q, const lcsa_kv_cache* kv, const int32_t* blk_idx,
+                                 const int32_t* blk_cnt, int32_t kmax, int32_t window, int32_t window_mode,
+                                 lcsa_tensor* o, float* lse, lcsa_stream_t stream) {
   lcsa_status s = check_tensor(q);
   if (s != LCSA_OK) return s;
   if ((s = check_cache(kv)) != LCSA_OK) return s;
@@ -675,6 +688,8 @@ lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_cache* kv, 
   p.nQB = p.nQT * p.Hb * p.Wb;
   p.kmax = kmax;
   p.cap = kv->cap_frames;
+  p.win = window;
+  p.win_mode = window_mode;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(q->D)));
   p.wait_limit_ns = g_wait_limit_ns;
   p.err = err;
@@ -688,6 +703,21 @@ lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_cache* kv, 
   else
     attn_fwd_kernel<64><<<static_cast<unsigned>(grid), ATTN_THREADS, AttnLayout<64>::SMEM_BYTES, cs>>>(tq, tk, tv, p);
   return launched();
+}
+
+lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_cache* kv, const int32_t* blk_idx,
+                                 const int32_t* blk_cnt, int32_t kmax, lcsa_tensor* o, float* lse,
+                                 lcsa_stream_t stream) {
+  return attn_fwd_impl(q, kv, blk_idx, blk_cnt, kmax, 0, LCSA_WINDOW_TRUNCATE_TOKENS, o, lse, stream);
+}
+
+lcsa_status lcsa_sparse_attn_fwd_window(const lcsa_tensor* q, const lcsa_kv_cache* kv, const int32_t* blk_idx,
+                                        const int32_t* blk_cnt, int32_t kmax, int32_t window, int32_t window_mode,
+                                        lcsa_tensor* o, float* lse, lcsa_stream_t stream) {
+  if (window < 0 || (window > 0 && window_mode != LCSA_WINDOW_TRUNCATE_TOKENS &&
+                     window_mode != LCSA_WINDOW_PRESERVE_TOKENS))
+    return LCSA_ERR_INVALID_ARG;
+  return attn_fwd_impl(q, kv, blk_idx, blk_cnt, kmax, window, window_mode, o, lse, stream);
 }
 
 lcsa_status lcsa_last_device_error(lcsa_stream_t stream) {

@@ -218,6 +218,22 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Token-level window along one axis of n tokens, seen from query token t:
+// w tokens with the query at offset w/2, clipped (mode 2) or shifted inward
+// (mode 3) at the frame edge.
+__host__ __device__ __forceinline__ void token_window(int t, int n, int w, int mode, int& lo, int& hi) {
+  const int s = t - w / 2;
+  if (mode == 2) {
+    lo = s > 0 ? s : 0;
+    hi = s + w < n ? s + w : n;
+  } else {
+    int st = s < n - w ? s : n - w;
+    st = st > 0 ? st : 0;
+    lo = st;
+    hi = st + w < n ? st + w : n;
+  }
+}
+
 // ---------------------------------------------------------------- math
 // 2^x on the special-function unit (PTX ex2.approx, flush-to-zero).
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -58,15 +58,28 @@ __device__ __forceinline__ double key_value(uint64_t k) {
   return __longlong_as_double(static_cast<long long>(u));
 }
 
-__device__ __forceinline__ void window_bounds(int i, int n, int w, int mode, int& lo, int& hi) {
+// Window of key blocks along one axis (n blocks) seen from query block i.
+// Modes 0 / 1: w blocks centred on the block, truncated / preserved at the
+// edge. Modes 2 / 3: the blocks holding a token that some token of block i
+// sees through its w-token window (truncated / preserved).
+__host__ __device__ __forceinline__ void window_bounds(int i, int n, int w, int mode, int& lo, int& hi) {
   if (w <= 0) { lo = 0; hi = n; return; }
+  if (mode >= 2) {
+    int a, b, c, d;
+    token_window(8 * i, 8 * n, w, mode, a, b);
+    token_window(8 * i + 7, 8 * n, w, mode, c, d);
+    lo = a / 8;
+    hi = (d - 1) / 8 + 1;
+    return;
+  }
   const int r = w / 2;
   if (mode == 0) {  // truncate at the frame edge
-    lo = max(0, i - r);
-    hi = min(n, i + r + 1);
+    lo = i - r > 0 ? i - r : 0;
+    hi = i + r + 1 < n ? i + r + 1 : n;
   } else {          // preserve: shift inward, keep w blocks
-    lo = max(0, min(i - r, n - w));
-    hi = min(n, lo + w);
+    int st = i - r < n - w ? i - r : n - w;
+    lo = st > 0 ? st : 0;
+    hi = lo + w < n ? lo + w : n;
   }
 }
 

@@ -77,7 +77,12 @@ typedef enum lcsa_status {
   LCSA_ERR_SCRATCH_LIMIT = -9  /* request exceeds the library's fixed scratch   */
 } lcsa_status;
 
-enum { LCSA_WINDOW_TRUNCATE = 0, LCSA_WINDOW_PRESERVE = 1 };
+enum {
+  LCSA_WINDOW_TRUNCATE = 0,         /* block window, clipped at the frame edge      */
+  LCSA_WINDOW_PRESERVE = 1,         /* block window, shifted inward at the edge      */
+  LCSA_WINDOW_TRUNCATE_TOKENS = 2,  /* token window, clipped at the frame edge      */
+  LCSA_WINDOW_PRESERVE_TOKENS = 3   /* token window, shifted inward at the edge      */
+};
 
 /* A token tensor [B][H][T][Y][X][D] of bf16 in device memory. */
 typedef struct lcsa_tensor {
@@ -121,11 +126,17 @@ typedef struct lcsa_kv_cache {
  *           0: keep K_i = min(C_i, max(1, ceil(density * C_i))) where C_i is
  *           the number of allowed (causal, in-window) key blocks of the row
  *           and density * C_i is a float64 product.
- * window    0: no window; else the odd side length of the square spatial
- *           window in blocks (radius window/2), centred on the query block.
- * window_mode  LCSA_WINDOW_TRUNCATE: clip the window at the frame edge;
- *           LCSA_WINDOW_PRESERVE: shift it inward so it always spans
- *           `window` blocks (start = max(0, min(y-r, Hb-window))).
+ * window    0: no window. Block modes: the odd side length of the square
+ *           spatial window in blocks (radius window/2), centred on the query
+ *           block. Token modes: the window's side in tokens (e.g. 72 for
+ *           1152 px): each query token t sees [t - window/2, t - window/2 +
+ *           window) per axis; a key block is a candidate when some token of
+ *           the query block sees some token of it, and the attention masks
+ *           each key token outside the query token's window
+ *           (lcsa_sparse_attn_fwd_window).
+ * window_mode  LCSA_WINDOW_TRUNCATE(_TOKENS): clip the window at the frame
+ *           edge; LCSA_WINDOW_PRESERVE(_TOKENS): shift it inward so it keeps
+ *           its width (start = max(0, min(c - window/2, n - window))).
  * tie_eps   near-tie band (1e-5): with tau the K_i-th largest score, blocks
  *           with score > tau+eps are kept and the remaining places go to the
  *           lowest-index blocks with tau-eps <= score <= tau+eps.
@@ -287,6 +298,25 @@ LCSA_API lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_ca
                                  const int32_t* blk_idx, const int32_t* blk_cnt,
                                  int32_t kmax, lcsa_tensor* o, float* lse,
                                  lcsa_stream_t stream);
+
+/*
+ * lcsa_sparse_attn_fwd_window - lcsa_sparse_attn_fwd with the token-level
+ * locality window (section 2.3: at inference each query's attention is limited
+ * to a local neighbourhood, e.g. 1152 x 1152 px = 72 x 72 tokens, with a
+ * boundary-truncate or boundary-preserve rule), applied inside the kept
+ * blocks: query token (y, x) sees key token (y', x') iff y' and x' lie in its
+ * window along each axis, [c - window/2, c - window/2 + window) clipped to the
+ * frame (LCSA_WINDOW_TRUNCATE_TOKENS) or shifted inward to keep its width
+ * (LCSA_WINDOW_PRESERVE_TOKENS). Use it with selections made with the same
+ * window and mode. A query token that sees no key of its kept blocks gets
+ * O = 0 and LSE = -inf. window = 0 is lcsa_sparse_attn_fwd. Other arguments
+ * and errors as lcsa_sparse_attn_fwd; LCSA_ERR_INVALID_ARG for a block-level
+ * window_mode with window > 0.
+ */
+LCSA_API lcsa_status lcsa_sparse_attn_fwd_window(const lcsa_tensor* q, const lcsa_kv_cache* kv,
+                                        const int32_t* blk_idx, const int32_t* blk_cnt,
+                                        int32_t kmax, int32_t window, int32_t window_mode,
+                                        lcsa_tensor* o, float* lse, lcsa_stream_t stream);
 
 /*
  * lcsa_segment_blocks - block lists for dense attention confined to one

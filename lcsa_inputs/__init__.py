@@ -39,6 +39,8 @@ __all__ = ["Workload", "WORKLOADS", "workload", "make_inputs", "small_variant"]
 
 WINDOW_TRUNCATE = 0
 WINDOW_PRESERVE = 1
+WINDOW_TRUNCATE_TOKENS = 2
+WINDOW_PRESERVE_TOKENS = 3
 
 
 @dataclass(frozen=True)
@@ -107,6 +109,13 @@ WORKLOADS = {
     "uhr_preserve": Workload("uhr_preserve", B=1, H=12, D=128, Y=96, X=168, q_frames=2,
                              kv_past=(4,), cap_frames=6, density=0.136, window=9,
                              window_mode=WINDOW_PRESERVE, seed=5),
+    # the same 1536x2688 frames with the window at token level: 72 x 72 tokens = 1152 x 1152 px
+    "uhr_truncate_tok": Workload("uhr_truncate_tok", B=1, H=12, D=128, Y=96, X=168, q_frames=2,
+                                 kv_past=(4,), cap_frames=6, density=0.136, window=72,
+                                 window_mode=WINDOW_TRUNCATE_TOKENS, seed=5),
+    "uhr_preserve_tok": Workload("uhr_preserve_tok", B=1, H=12, D=128, Y=96, X=168, q_frames=2,
+                                 kv_past=(4,), cap_frames=6, density=0.136, window=72,
+                                 window_mode=WINDOW_PRESERVE_TOKENS, seed=5),
 }
 
 
