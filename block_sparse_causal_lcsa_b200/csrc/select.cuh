@@ -123,6 +123,32 @@ score_kernel(const __grid_constant__ SelectParams p) {
   const int ncur = min(SC_CANDS, g.ncand - c0);
   const int tid = threadIdx.x;
 
+  // With a window, most (row, candidate) pairs of a CTA can lie outside every
+  // row's window: a CTA none of whose pairs is inside only writes key 0.
+  if (p.window > 0) {
+    bool any = false;
+    const int cand = tid % SC_CANDS;
+    if (cand < ncur) {
+      const int spk = (c0 + cand) % HbWb;
+      const int yk = spk / p.Wb, xk = spk - yk * p.Wb;
+      for (int r = tid / SC_CANDS; r < nrows; r += SC_THREADS / SC_CANDS) {
+        const int sp = sp0 + r;
+        int y0, y1, x0, x1;
+        window_bounds(sp / p.Wb, p.Hb, p.window, p.window_mode, y0, y1);
+        window_bounds(sp % p.Wb, p.Wb, p.window, p.window_mode, x0, x1);
+        any |= yk >= y0 && yk < y1 && xk >= x0 && xk < x1;
+      }
+    }
+    if (!__syncthreads_or(any)) {
+      for (int e = tid; e < nrows * SC_CANDS; e += SC_THREADS) {
+        const int r = e / SC_CANDS, c = e % SC_CANDS;
+        if (c < ncur)
+          p.keys[(static_cast<int64_t>(bh) * nQB + tq * HbWb + sp0 + r) * p.c_stride + c0 + c] = 0ull;
+      }
+      return;
+    }
+  }
+
   const int warp = tid >> 5, lane = tid & 31;
   constexpr int V2 = D / 2;                       // 16-byte vectors per pooled row
   constexpr int PER_LANE = V2 / 32;               // vectors per lane per row
