@@ -158,24 +158,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int nkb = static_cast<int>((end >> 1) - m_first) * HbWb;  // valid block ids
   const int fq0 = p.Tq - 2 * p.nQT + 2 * tq;   // older frame of the query block (-1: missing)
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < B_COUNT; ++i)
-      mbar_init(bar(i), (i >= B_P_FULL && i < B_P_FULL + S_BUFS) ? SOFTMAX_THREADS : 1u);
-    *abort_flag = 0;
-    mbar_init_fence();
-    tma_prefetch_map(&tmQ);
-    tma_prefetch_map(&tmK);
-    tma_prefetch_map(&tmV);
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
-  }
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const WaitCtx w{p.wait_limit_ns, abort_flag, p.err};
-
   auto checked = [&](int blk) -> int {
     if (blk < 0 || blk >= nkb) {
       atomicOr(p.err, DEVERR_BOUNDS);
@@ -183,7 +165,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     return blk;
   };
-
   // One 128-token tile = 2 frames x D/64 channel columns of 8 KB boxes.
   auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar_full, int x8, int y8,
                        int fr0, int fr1) {
@@ -205,15 +186,40 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     y8 = 8 * (spk / p.Wb);
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ Q + K producer
-    if (lane == 0 && n > 0) {
+  if (threadIdx.x == 0) {
+    // thread 0 is also the Q/K producer: it initialises the barriers and starts
+    // the Q and first K copies right away, so their latency overlaps the
+    // tensor-memory allocation and the CTA-wide barrier
+    const int first_blk = blist[0];              // row capacity kmax >= 1
+    for (int i = 0; i < B_COUNT; ++i)
+      mbar_init(bar(i), (i >= B_P_FULL && i < B_P_FULL + S_BUFS) ? SOFTMAX_THREADS : 1u);
+    *abort_flag = 0;
+    mbar_init_fence();
+    if (n > 0) {
       mbar_arrive_expect_tx(bar(B_Q_FULL), L::TILE_BYTES);
       // a missing older query frame is replaced by the newer one (rows not stored)
       load_tile(&tmQ, sbase + L::OFF_Q, bar(B_Q_FULL), 8 * xq, 8 * yq, fq0 < 0 ? fq0 + 1 : fq0, fq0 + 1);
-      int issued_k = 0;
-      int next_blk = checked(blist[0]);
-      for (int j = 0; j < n; ++j) {
+      int x8, y8, s0, s1;
+      tile_coords(checked(first_blk), x8, y8, s0, s1);
+      mbar_arrive_expect_tx(bar(B_K_FULL), L::TILE_BYTES);
+      load_tile(&tmK, sbase + L::OFF_K, bar(B_K_FULL), x8, y8, s0, s1);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx w{p.wait_limit_ns, abort_flag, p.err};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ Q + K producer
+    if (lane == 0 && n > 0) {
+      int issued_k = 1;                           // Q and K_0 went out before the CTA barrier
+      int next_blk = n > 1 ? checked(blist[1]) : 0;
+      for (int j = 1; j < n; ++j) {
         const int blk = next_blk;
         if (j + 1 < n) next_blk = checked(blist[j + 1]);
         int x8, y8, s0, s1;
