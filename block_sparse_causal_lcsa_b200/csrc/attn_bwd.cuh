@@ -15,8 +15,9 @@
 //                     (the transpose of the selection), one warp per key block.
 //   bwd_dq_kernel     one CTA per query block over its kept key blocks: S and
 //                     dP (tcgen05, shared-memory operands) into tensor memory,
-//                     dS in bf16 written back over dP, dQ += dS K (dS from
-//                     tensor memory).
+//                     dS in bf16 into its own tensor-memory columns, dQ += dS K
+//                     (dS from tensor memory) issued after the next block's S
+//                     and dP so that it overlaps the next elementwise step.
 //   bwd_dkdv_kernel   one CTA per key block over the query blocks that kept
 //                     it: S^T = K Q^T and dP^T = V dO^T, P^T and dS^T in bf16
 //                     written back over them, dV += P^T dO and dK += dS^T Q, both
@@ -197,12 +198,13 @@ __device__ __forceinline__ void bwd_load_tile(const CUtensorMap* map, uint32_t d
 }
 
 // Elementwise step of one 128x128 tile, one row per thread: P = 2^(S*scale_log2
-// - lse2), G = P (dP - delta), both rounded to bf16 and written back in place
-// over the first 64 columns of their own buffers (column chunk c of 32 values
-// packs into columns [16c, 16c+16), which chunk c has already read). The column
-// vectors lse2 / delta (or per-row scalars) and the masks come from the caller.
+// - lse2), G = P (dP - delta), both rounded to bf16; P is written back in place
+// over the first 64 columns of S and G to the 64 columns at t_g (t_g = t_dp
+// writes it in place too: column chunk c of 32 values packs into columns
+// [16c, 16c+16), which chunk c has already read). The column vectors lse2 /
+// delta (or per-row scalars) and the masks come from the caller.
 template <bool COL_VECTORS>
-__device__ __forceinline__ void bwd_tile_elementwise(uint32_t t_s, uint32_t t_dp, float scale_log2,
+__device__ __forceinline__ void bwd_tile_elementwise(uint32_t t_s, uint32_t t_dp, uint32_t t_g, float scale_log2,
                                                      const float* lse2v, const float* deltav, float lse2_row,
                                                      float delta_row, bool zero_cols_lo, bool zero_row,
                                                      bool write_p) {
@@ -230,12 +232,14 @@ __device__ __forceinline__ void bwd_tile_elementwise(uint32_t t_s, uint32_t t_dp
       gg[k] = pack_bf16x2(gv[0], gv[1]);
     }
     if (write_p) tmem_st_32x32b_x16(t_s + c * 16, pp);
-    tmem_st_32x32b_x16(t_dp + c * 16, gg);
+    tmem_st_32x32b_x16(t_g + c * 16, gg);
   }
   tmem_st_wait();
 }
 
 // ---------------------------------------------------------------- dQ
+constexpr uint32_t DS_COL = 256;   // dS (bf16 pairs, 64 columns) of the dQ kernel
+constexpr uint32_t DQ_COL = 384;   // dQ accumulator of the dQ kernel
 enum : int {
   DQB_QD_FULL = 0,      // Q and dO of the block
   DQB_K_FULL = 1,       // 2
@@ -292,7 +296,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   }
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;          // S: cols 0-127, dP/dS: 128-255, dQ: 256-383
+  const uint32_t tmem = *tmem_slot;          // S: cols 0-127, dP: 128-255, dS: 256-319, dQ: 384-511
   const WaitCtx w{p.wait_limit_ns, abort_flag, p.err};
   auto checked = [&](int blk) -> int {
     if (blk < 0 || blk >= nkb) {
@@ -338,12 +342,27 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       constexpr uint32_t ID_SS = idesc_bf16_f32(128, 128, false);   // S, dP: K-major A and B
       constexpr uint32_t ID_DQ = idesc_bf16_f32(128, D, true);      // dQ: B = K, channels contiguous
       bool ok = wait_bounded(bar(DQB_QD_FULL), 0, w);
+      // dQ += dS K for block j-1 (dS in its own tensor-memory columns) is issued
+      // right after S_j and dP_j, so it runs while the elementwise warps work on
+      // block j.
+      auto issue_dq = [&](int jj) {
+        const uint32_t ka = sbase + L::DQ_K + (jj & 1) * L::TILE;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          // A = dS (16 keys = 8 packed columns), B = K: 16 keys = 16 rows of 128 bytes,
+          // 64-channel columns 16 KB apart
+          bwd_umma_ts(tmem + DQ_COL, tmem + DS_COL + kk * 8, desc_sw128(ka + kk * 2048, L::CHUNK, 1024), ID_DQ,
+                      (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar(DQB_DQ_DONE));
+        umma_commit(bar(DQB_K_EMPTY + (jj & 1)));
+      };
       for (int j = 0; ok && j < n; ++j) {
         const int st = j & 1;
         if (!(ok = wait_bounded(bar(DQB_K_FULL + st), (j >> 1) & 1, w))) break;
         if (!(ok = wait_bounded(bar(DQB_V_FULL + st), (j >> 1) & 1, w))) break;
-        // S and dP overwrite the buffers of block j-1: its dQ MMA must be done
-        if (j > 0 && !(ok = wait_bounded(bar(DQB_DQ_DONE), (j - 1) & 1, w))) break;
+        // S_j and dP_j overwrite what the elementwise warps read for block j-1
+        if (j > 0 && !(ok = wait_bounded(bar(DQB_G_FULL), (j - 1) & 1, w))) break;
         tc_fence_after();
         const uint32_t ka = sbase + L::DQ_K + st * L::TILE, va = sbase + L::DQ_V + st * L::TILE;
 #pragma unroll
@@ -360,17 +379,11 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
         umma_commit(bar(DQB_SD_FULL));
         umma_commit(bar(DQB_V_EMPTY + st));
-        if (!(ok = wait_bounded(bar(DQB_G_FULL), j & 1, w))) break;
+        if (j > 0) issue_dq(j - 1);
+      }
+      if (ok && (ok = wait_bounded(bar(DQB_G_FULL), (n - 1) & 1, w))) {
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          // A = dS (16 keys = 8 packed columns), B = K: 16 keys = 16 rows of 128 bytes,
-          // 64-channel columns 16 KB apart
-          bwd_umma_ts(tmem + 256, tmem + 128 + kk * 8, desc_sw128(ka + kk * 2048, L::CHUNK, 1024), ID_DQ,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(bar(DQB_DQ_DONE));
-        umma_commit(bar(DQB_K_EMPTY + st));
+        issue_dq(n - 1);
       }
       umma_commit(bar(DQB_DRAIN));
       bwd_drain_wait(bar(DQB_DRAIN), 0, w.limit_ns);
@@ -387,9 +400,11 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     for (int j = 0; j < n; ++j) {
       const bool partial = oldest_partial && checked(blist[j]) < HbWb;  // keys 0-63 absent
       if (!bwd_warp_wait(bar(DQB_SD_FULL), j & 1, w)) { done = false; break; }
+      // the dS columns are free once dQ of block j-1 (their last reader) is done
+      if (j > 0 && !bwd_warp_wait(bar(DQB_DQ_DONE), (j - 1) & 1, w)) { done = false; break; }
       tc_fence_after();
-      bwd_tile_elementwise<false>(t_lane, t_lane + 128, p.scale_log2, nullptr, nullptr, lse2, delta, partial,
-                                  false, false);
+      bwd_tile_elementwise<false>(t_lane, t_lane + 128, t_lane + DS_COL, p.scale_log2, nullptr, nullptr, lse2, delta,
+                                  partial, false, false);
       tc_fence_before();
       mbar_arrive(bar(DQB_G_FULL));
     }
@@ -404,7 +419,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t g[32];
         if (n > 0) {
-          tmem_ld_32x32b_x32(t_lane + 256 + c0, g);
+          tmem_ld_32x32b_x32(t_lane + DQ_COL + c0, g);
           tmem_ld_wait();
         } else {
 #pragma unroll
@@ -580,8 +595,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (!bwd_warp_wait(bar(KVB_SD_FULL), j & 1, w)) { done = false; break; }
       tc_fence_after();
       const float* vec = reinterpret_cast<const float*>(smem + L::KV_VEC + st * 1024);
-      bwd_tile_elementwise<true>(t_lane, t_lane + 128, p.scale_log2, vec, vec + 128, 0.f, 0.f, false, zero_row,
-                                 true);
+      bwd_tile_elementwise<true>(t_lane, t_lane + 128, t_lane + 128, p.scale_log2, vec, vec + 128, 0.f, 0.f, false,
+                                 zero_row, true);
       tc_fence_before();
       mbar_arrive(bar(KVB_G_FULL));
     }
