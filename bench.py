@@ -1,15 +1,22 @@
 """Benchmark: one streaming LCSA step per 8-frame chunk at 768x1408 on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload chunk|multistream|uhr_truncate|uhr_preserve|clip|clip_5|clip_30]
+                    [--workload chunk|multistream|uhr_truncate|uhr_preserve|uhr_truncate_tok|
+                                uhr_preserve_tok|clip|clip_5|clip_30]
+                    [--mode fwd|bwd|segment]
 
-A step is the whole hot path over one chunk: lcsa_pool_qk (Q and the new K),
-lcsa_kv_append (K, V, pooled K into the ring cache, evicting the oldest
-frames), lcsa_select_blocks (coarse map, causal mask, top-K) and
-lcsa_sparse_attn_fwd, with Q/K/V resident in HBM. L2 is flushed (a 512 MB
-write) before every timed step, outside the timed events. Under torchrun each
-rank streams its own independent video (weak scaling, no data-path
-collective); the step time is the max over ranks.
+A step is the whole hot path over one chunk: lcsa_pool_qk (Q), lcsa_kv_append
+(K, V and K pooled on the way into the ring cache, evicting the oldest frames),
+lcsa_select_blocks (coarse map, causal mask, top-K) and lcsa_sparse_attn_fwd,
+with Q/K/V resident in HBM. L2 is flushed (a 512 MB write and a 256 MB read)
+before every timed step, outside the timed events. The step is timed twice:
+eagerly with CUDA events between the kernels (the per-kernel split) and
+replayed from a CUDA graph (the headline value: the same kernels and work,
+one launch). Under torchrun each rank streams its own independent video (weak
+scaling, no data-path collective); the step time is the max over ranks.
+
+--mode bwd times the attention backward on a whole clip (training form);
+--mode segment the stage-1 dense segment attention, forward and backward.
 
 Rank 0 prints one JSON line. `--impl reference` times the fp64 CPU oracle on
 a bounded sample of the same workload instead (rank 0 only).
@@ -380,6 +387,28 @@ def run_ours(args, world, rank, local):
     if lc.last_device_error() != 0:
         raise RuntimeError("device error during the end-to-end steps")
 
+    # the same step replayed from a CUDA graph (one launch per step), inputs in
+    # the graph's static buffers, L2 flushed outside the timed events
+    graph = None
+    if streaming:
+        step.cache.set_state(base_state)
+        step.graph_step(*chunks[0])
+        g_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for i in range(args.warmup + args.steps):
+            flush_l2()
+            step.cache.set_state(base_state)
+            if i >= args.warmup:
+                g_ev[i - args.warmup][0].record()
+            step.graph_step()
+            if i >= args.warmup:
+                g_ev[i - args.warmup][1].record()
+        torch.cuda.synchronize()
+        if lc.last_device_error() != 0:
+            raise RuntimeError("device error during the graph steps")
+        g_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in g_ev), world)
+        graph = {"ms_per_chunk": round(whole_job_ms_per_chunk(g_ms, chunks_per_step, world), 4),
+                 "graph_launches_per_step": 1}
+
     # HBM-side kernels: algorithmic bytes per launch
     tokens_q = w.B * w.H * q_frames_step * w.Y * w.X
     if "kv_append" in per_kernel:
@@ -402,9 +431,18 @@ def run_ours(args, world, rank, local):
         if rec.get("source_hash", "").strip() == attn_source_hash():
             traffic = int(rec["bytes_per_launch"])
 
+    # the headline is the step as a user runs it in production: replayed from a
+    # CUDA graph (same kernels, same work, one launch); the eager run with CUDA
+    # events between the kernels gives the per-kernel split
+    eager_value = value
+    step_ms = mean_step_max
+    if graph is not None:
+        value = graph["ms_per_chunk"]
+        step_ms = value * chunks_per_step * world
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(mean_step_max, 4),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+        "eager_ms_per_chunk": round(eager_value, 4),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16, shapes of the pages' 768x1408 workload)",
         "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload,
@@ -421,6 +459,7 @@ def run_ours(args, world, rank, local):
                      "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % peaks["source"],
                      "flops_per_launch": flops, "traffic": traffic},
         "hbm_kernels": {k2: round(v2, 1) for k2, v2 in hbm.items()},
+        "cuda_graph": graph,
         "hbm_peak_gbs": peaks["hbm_gbs"],
         "e2e": e2e,
         "gpu_launches": len(kernels) * args.steps,

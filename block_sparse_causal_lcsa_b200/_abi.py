@@ -66,6 +66,7 @@ PROTOTYPES = {
                                C.c_void_p]),
     "lcsa_kv_append": (C.c_int, [C.POINTER(KVCacheStruct), C.POINTER(Tensor), C.POINTER(Tensor),
                                  C.c_void_p, C.c_int32, C.c_void_p]),
+    "lcsa_kv_advance": (C.c_int, [C.POINTER(KVCacheStruct), C.c_int32, C.c_int32, C.c_int32]),
     "lcsa_select_kmax": (C.c_int32, [C.POINTER(KVCacheStruct), C.c_int32,
                                      C.POINTER(SelectParamsStruct)]),
     "lcsa_select_workspace_bytes": (C.c_size_t, [C.POINTER(KVCacheStruct), C.c_int32]),

@@ -347,6 +347,45 @@ class StreamingStep:
         self.blk_cnt = torch.empty((B, H, nQB), dtype=torch.int32, device=dev)
         self.o = torch.empty((B, H, q_frames, Y, X, D), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((B, H, q_frames, Y, X), dtype=torch.float32, device=dev)
+        self._static = None
+        self._graphs = {}
+
+    def graph_step(self, q: Optional[torch.Tensor] = None, k_new: Optional[torch.Tensor] = None,
+                   v_new: Optional[torch.Tensor] = None):
+        """The same step replayed from a CUDA graph: the inputs are copied into
+        static buffers (without inputs, the buffers are used as they are: the
+        caller may have written the chunk there), then one graph launch runs
+        pool, append, select and attention. The library passes frame numbers to its kernels modulo the
+        ring capacity, so a stream in steady state needs one graph per ring
+        phase; each is captured the first time its phase comes up (make that
+        first step an ordinary one outside any timing). Returns (o, lse), the
+        step's static output buffers."""
+        if self._static is None:
+            if q is None:
+                raise ValueError("the first graph_step needs the chunk")
+            self._static = (torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new))
+            self._graphs = {}
+        sq, sk, sv = self._static
+        if q is not None:
+            sq.copy_(q)
+            sk.copy_(k_new)
+            sv.copy_(v_new)
+        cap = self.cache.cap_frames
+        key = tuple((b % cap, e - b) for b, e in self.cache.state())
+        g = self._graphs.get(key)
+        if g is None:
+            saved = self.cache.state()
+            self(sq, sk, sv)                  # device set-up and a warm run outside the capture
+            torch.cuda.synchronize()
+            self.cache.set_state(saved)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self(sq, sk, sv)
+            self.cache.set_state(saved)       # the capture advanced the host state without running
+            self._graphs[key] = g
+        g.replay()
+        _check(_lib.lcsa_kv_advance(C.byref(self.cache.struct), sk.shape[2], sk.shape[0], 0), "lcsa_kv_advance")
+        return self.o, self.lse
 
     def __call__(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
                  stream: Optional[torch.cuda.Stream] = None):

@@ -215,6 +215,29 @@ lcsa_status launch_ingest(const IngestParams& p, int D, cudaStream_t cs) {
   return launched();
 }
 
+// Frame numbers as the kernels see them: shifted down by whole multiples of the
+// ring capacity. Ring slots (a % cap, m % (cap/2) with cap even), the parity of
+// begin and all lengths are unchanged, so the launches of a steady stream
+// repeat with the period of the ring and can be replayed from a CUDA graph.
+int64_t ring_base(int64_t begin, int cap) { return begin >= 0 ? begin - begin % cap : 0; }
+
+// Cache state after appending Tn frames to streams [offset, offset+n): the
+// absolute frame of the chunk's first frame, and the new begin / end.
+lcsa_status append_state(const lcsa_kv_cache* kv, int Tn, int n, int offset, int64_t* first, int64_t* nb,
+                         int64_t* ne) {
+  for (int bn = 0; bn < n; ++bn) {
+    const int b = bn + offset;
+    const bool empty = kv->end[b] == kv->begin[b];
+    if (!empty && (Tn & 1)) return LCSA_ERR_SHAPE;  // odd chunks only start a stream
+    first[bn] = empty ? kv->end[b] + (Tn & 1) : kv->end[b];
+    const int64_t e = first[bn] + Tn;
+    const int64_t old_begin = empty ? first[bn] : kv->begin[b];
+    ne[bn] = e;
+    nb[bn] = old_begin > e - kv->cap_frames ? old_begin : e - kv->cap_frames;
+  }
+  return LCSA_OK;
+}
+
 }  // namespace
 }  // namespace lcsa
 
@@ -286,18 +309,9 @@ lcsa_status lcsa_kv_append(lcsa_kv_cache* kv, const lcsa_tensor* k_new, const lc
   const int Tn = kn->T;
   const int cap = kv->cap_frames;
   AppendParams p{};
-  int64_t new_begin[LCSA_MAX_STREAMS], new_end[LCSA_MAX_STREAMS];
-  for (int bn = 0; bn < kn->B; ++bn) {
-    const int b = bn + stream_offset;
-    const bool empty = kv->end[b] == kv->begin[b];
-    if (!empty && (Tn & 1)) return LCSA_ERR_SHAPE;  // odd chunks only start a stream
-    const int64_t first = empty ? kv->end[b] + (Tn & 1) : kv->end[b];
-    const int64_t e = first + Tn;
-    const int64_t old_begin = empty ? first : kv->begin[b];
-    new_end[bn] = e;
-    new_begin[bn] = old_begin > e - cap ? old_begin : e - cap;
-    p.first_abs[bn] = first;
-  }
+  int64_t new_begin[LCSA_MAX_STREAMS], new_end[LCSA_MAX_STREAMS], first[LCSA_MAX_STREAMS];
+  if ((s = append_state(kv, Tn, kn->B, stream_offset, first, new_begin, new_end)) != LCSA_OK) return s;
+  for (int bn = 0; bn < kn->B; ++bn) p.first_abs[bn] = first[bn] - ring_base(first[bn], cap);
   // Every stream of one call appends the same frames of the chunk: the newest
   // min(Tn, cap) frames (cap is even, so the kept blocks are whole or the
   // chunk's own one-frame oldest block).
@@ -362,6 +376,20 @@ lcsa_status lcsa_kv_append(lcsa_kv_cache* kv, const lcsa_tensor* k_new, const lc
   for (int bn = 0; bn < kn->B; ++bn) {
     kv->begin[bn + stream_offset] = new_begin[bn];
     kv->end[bn + stream_offset] = new_end[bn];
+  }
+  return LCSA_OK;
+}
+
+lcsa_status lcsa_kv_advance(lcsa_kv_cache* kv, int32_t frames, int32_t n_streams, int32_t stream_offset) {
+  lcsa_status s = check_cache(kv);
+  if (s != LCSA_OK) return s;
+  if (frames < 1 || n_streams < 1 || stream_offset < 0 || stream_offset + n_streams > kv->B)
+    return LCSA_ERR_INVALID_ARG;
+  int64_t first[LCSA_MAX_STREAMS], nb[LCSA_MAX_STREAMS], ne[LCSA_MAX_STREAMS];
+  if ((s = append_state(kv, frames, n_streams, stream_offset, first, nb, ne)) != LCSA_OK) return s;
+  for (int bn = 0; bn < n_streams; ++bn) {
+    kv->begin[bn + stream_offset] = nb[bn];
+    kv->end[bn + stream_offset] = ne[bn];
   }
   return LCSA_OK;
 }
@@ -442,7 +470,11 @@ lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames, const lcs
   p.tie_eps = sp->tie_eps;
   p.sqrt_d = std::sqrt(static_cast<double>(kv->D));
   p.err = err;
-  for (int b = 0; b < kv->B; ++b) { p.kv_begin[b] = kv->begin[b]; p.kv_end[b] = kv->end[b]; }
+  for (int b = 0; b < kv->B; ++b) {
+    const int64_t base = ring_base(kv->begin[b], kv->cap_frames);
+    p.kv_begin[b] = kv->begin[b] - base;
+    p.kv_end[b] = kv->end[b] - base;
+  }
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const dim3 sgrid(static_cast<unsigned>((c_stride + SC_CANDS - 1) / SC_CANDS),
                    static_cast<unsigned>((HbWb + SC_ROWS - 1) / SC_ROWS),
@@ -491,7 +523,11 @@ lcsa_status lcsa_segment_blocks(int32_t q_frames, const lcsa_kv_cache* kv, int32
   p.HbWb = (kv->Y / 8) * (kv->X / 8);
   p.kmax = kmax;
   p.rows = rows;
-  for (int b = 0; b < kv->B; ++b) { p.kv_begin[b] = kv->begin[b]; p.kv_end[b] = kv->end[b]; }
+  for (int b = 0; b < kv->B; ++b) {
+    const int64_t base = ring_base(kv->begin[b], kv->cap_frames);
+    p.kv_begin[b] = kv->begin[b] - base;
+    p.kv_end[b] = kv->end[b] - base;
+  }
   // one warp per query-block row, rows numbered bh * nQB + qb
   segment_blocks_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0,
                           static_cast<cudaStream_t>(stream)>>>(p);
@@ -596,7 +632,11 @@ lcsa_status lcsa_sparse_attn_bwd(const lcsa_tensor* q, const lcsa_kv_cache* kv, 
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(q->D)));
   p.wait_limit_ns = g_wait_limit_ns;
   p.err = err;
-  for (int b = 0; b < kv->B; ++b) { p.kv_begin[b] = kv->begin[b]; p.kv_end[b] = kv->end[b]; }
+  for (int b = 0; b < kv->B; ++b) {
+    const int64_t base = ring_base(kv->begin[b], kv->cap_frames);
+    p.kv_begin[b] = kv->begin[b] - base;
+    p.kv_end[b] = kv->end[b] - base;
+  }
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const unsigned n_q = static_cast<unsigned>(z.BH * z.nQB), n_k = static_cast<unsigned>(z.BH * z.nKBmax);
   if (q->D == 128) {
@@ -693,7 +733,11 @@ static lcsa_status attn_fwd_impl(const lcsa_tensor* q, const lcsa_kv_cache* kv, 
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(q->D)));
   p.wait_limit_ns = g_wait_limit_ns;
   p.err = err;
-  for (int b = 0; b < kv->B; ++b) { p.kv_begin[b] = kv->begin[b]; p.kv_end[b] = kv->end[b]; }
+  for (int b = 0; b < kv->B; ++b) {
+    const int64_t base = ring_base(kv->begin[b], kv->cap_frames);
+    p.kv_begin[b] = kv->begin[b] - base;
+    p.kv_end[b] = kv->end[b] - base;
+  }
   const int64_t grid = static_cast<int64_t>(q->B) * q->H * p.nQB;  // one CTA per query block
   if (grid > 0x7fffffff) return LCSA_ERR_SHAPE;
   if (grid == 0) return LCSA_OK;

@@ -193,6 +193,19 @@ LCSA_API lcsa_status lcsa_kv_append(lcsa_kv_cache* kv, const lcsa_tensor* k_new,
                            int32_t stream_offset, lcsa_stream_t stream);
 
 /*
+ * lcsa_kv_advance - the host-side part of lcsa_kv_append alone: advance the
+ * begin / end of streams [stream_offset, stream_offset + n_streams) as
+ * appending `frames` frames would, launching nothing. For replaying a
+ * captured CUDA graph of a streaming step: the graph performs the device
+ * writes, this call keeps the cache state in step. The library passes frame
+ * numbers to its kernels shifted down by whole multiples of cap_frames, so
+ * the launches of a stream in steady state repeat every cap_frames / frames
+ * steps. Same errors as lcsa_kv_append's state checks.
+ */
+LCSA_API lcsa_status lcsa_kv_advance(lcsa_kv_cache* kv, int32_t frames, int32_t n_streams,
+                            int32_t stream_offset);
+
+/*
  * Row capacity blk_idx needs for a selection with these parameters over the
  * cache's current state and q_frames query frames (the largest K_i).
  * Returns 0 on invalid arguments.

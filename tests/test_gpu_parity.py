@@ -173,6 +173,31 @@ def test_streaming_sequence_with_eviction(lc):
             check_output(o[0, h].double().cpu().numpy(), ref["O"], lse[0, h].double().cpu().numpy(), ref["LSE"])
 
 
+def test_graph_replay_equals_eager_steps(lc):
+    """Eight 2-frame chunks through a 6-frame cache, eagerly and from CUDA graphs
+    (one per ring phase): identical outputs, cache contents and state."""
+    w = li.Workload("graph", B=2, H=2, D=128, Y=16, X=24, q_frames=2, kv_past=(0, 0), cap_frames=6,
+                    density=0.4, seed=91)
+    caches = [lc.KVCache(w.B, w.H, w.cap_frames, w.Y, w.X, w.D) for _ in range(2)]
+    for c in caches:
+        c.k.zero_(), c.v.zero_(), c.k_pool.zero_()
+    steps = [lc.StreamingStep(c, 2, params_of(lc, w)) for c in caches]
+    g = torch.Generator().manual_seed(7)
+    for t in range(8):
+        q, k, v = (torch.randn((w.B, w.H, 2, w.Y, w.X, w.D), generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+        o0, l0 = steps[0](q, k, v)
+        o1, l1 = steps[1].graph_step(q, k, v)
+        torch.cuda.synchronize()
+        assert lc.last_device_error() == 0
+        assert torch.equal(o0, o1) and torch.equal(l0, l1), "step %d" % t
+        assert caches[0].state() == caches[1].state()
+    assert torch.equal(caches[0].k, caches[1].k) and torch.equal(caches[0].v, caches[1].v)
+    assert torch.equal(caches[0].k_pool, caches[1].k_pool)
+    # filling states (empty, 2, 4 frames), then the three phases of a full ring,
+    # which steps 7 and 8 replay
+    assert len(steps[1]._graphs) == 6
+
+
 @pytest.mark.parametrize("first,q_frames", [(1, 1), (3, 3), (5, 2)])
 def test_odd_first_chunk_partial_blocks(lc, first, q_frames):
     """A stream whose first chunk has an odd frame count: the oldest key block
