@@ -14,6 +14,7 @@ from .api import (  # noqa: F401
     WINDOW_PRESERVE_TOKENS,
     WINDOW_TRUNCATE,
     WINDOW_TRUNCATE_TOKENS,
+    attn_workspace,
     debug_exp2_poly,
     debug_set_wait_limit_ns,
     debug_stalled_wait,

@@ -82,6 +82,10 @@ PROTOTYPES = {
     "lcsa_sparse_attn_fwd_window": (C.c_int, [C.POINTER(Tensor), C.POINTER(KVCacheStruct), C.c_void_p, C.c_void_p,
                                               C.c_int32, C.c_int32, C.c_int32, C.POINTER(Tensor), C.c_void_p,
                                               C.c_void_p]),
+    "lcsa_sparse_attn_fwd_workspace_bytes": (C.c_size_t, [C.c_int32]),
+    "lcsa_sparse_attn_fwd_ex": (C.c_int, [C.POINTER(Tensor), C.POINTER(KVCacheStruct), C.c_void_p, C.c_void_p,
+                                          C.c_int32, C.c_int32, C.c_int32, C.POINTER(Tensor), C.c_void_p,
+                                          C.c_void_p, C.c_size_t, C.c_void_p]),
     "lcsa_segment_kmax": (C.c_int32, [C.POINTER(KVCacheStruct)]),
     "lcsa_segment_blocks": (C.c_int, [C.c_int32, C.POINTER(KVCacheStruct), C.c_int32, C.c_void_p, C.c_void_p,
                                       C.c_void_p]),

@@ -219,10 +219,13 @@ def select_blocks_noalloc(q_pool: torch.Tensor, q_frames: int, cache: KVCache, p
 def sparse_attn_fwd(q: torch.Tensor, cache: KVCache, blk_idx: torch.Tensor, blk_cnt: torch.Tensor,
                     o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                     with_lse: bool = True, stream: Optional[torch.cuda.Stream] = None,
-                    window: int = 0, window_mode: int = WINDOW_TRUNCATE_TOKENS):
+                    window: int = 0, window_mode: int = WINDOW_TRUNCATE_TOKENS,
+                    workspace: Optional[torch.Tensor] = None):
     """Attention of the query chunk over its kept key blocks: (O bf16 like q, LSE fp32).
     With ``window`` > 0 (a token-level window mode), each query token only sees
-    the key tokens inside its window (lcsa_sparse_attn_fwd_window)."""
+    the key tokens inside its window. With a ``workspace`` (see
+    attn_workspace), a partly empty last wave of CTAs is evened out by splitting
+    its query blocks in two (lcsa_sparse_attn_fwd_ex)."""
     if o is None:
         o = torch.empty_like(q)
     if lse is None and with_lse:
@@ -231,7 +234,13 @@ def sparse_attn_fwd(q: torch.Tensor, cache: KVCache, blk_idx: torch.Tensor, blk_
         raise ValueError("blk_idx and blk_cnt must be contiguous")
     qd, od = tensor_desc(q), tensor_desc(o)
     lse_ptr = lse.data_ptr() if lse is not None else None
-    if window > 0:
+    if workspace is not None:
+        _check(_lib.lcsa_sparse_attn_fwd_ex(C.byref(qd), C.byref(cache.struct), blk_idx.data_ptr(),
+                                            blk_cnt.data_ptr(), blk_idx.shape[-1], window, window_mode,
+                                            C.byref(od), lse_ptr, workspace.data_ptr(),
+                                            workspace.numel() * workspace.element_size(), _stream(stream)),
+               "lcsa_sparse_attn_fwd_ex")
+    elif window > 0:
         _check(_lib.lcsa_sparse_attn_fwd_window(C.byref(qd), C.byref(cache.struct), blk_idx.data_ptr(),
                                                 blk_cnt.data_ptr(), blk_idx.shape[-1], window, window_mode,
                                                 C.byref(od), lse_ptr, _stream(stream)),
@@ -242,6 +251,12 @@ def sparse_attn_fwd(q: torch.Tensor, cache: KVCache, blk_idx: torch.Tensor, blk_
                                          _stream(stream)),
                "lcsa_sparse_attn_fwd")
     return o, lse
+
+
+def attn_workspace(head_dim: int, device="cuda") -> torch.Tensor:
+    """Workspace for sparse_attn_fwd's tail split (lcsa_sparse_attn_fwd_workspace_bytes)."""
+    n = int(_lib.lcsa_sparse_attn_fwd_workspace_bytes(head_dim))
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
 
 
 def segment_blocks(q_frames: int, cache: KVCache, kmax: Optional[int] = None,
@@ -347,6 +362,7 @@ class StreamingStep:
         self.blk_cnt = torch.empty((B, H, nQB), dtype=torch.int32, device=dev)
         self.o = torch.empty((B, H, q_frames, Y, X, D), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((B, H, q_frames, Y, X), dtype=torch.float32, device=dev)
+        self.attn_ws = attn_workspace(D, dev)
         self._static = None
         self._graphs = {}
 
@@ -395,5 +411,5 @@ class StreamingStep:
                       self.blk_idx, self.blk_cnt, self.workspace, stream)
         tw = self.params.window if self.params.window_mode >= WINDOW_TRUNCATE_TOKENS else 0
         sparse_attn_fwd(q, self.cache, self.blk_idx, self.blk_cnt, self.o, self.lse, stream=stream,
-                        window=tw, window_mode=self.params.window_mode)
+                        window=tw, window_mode=self.params.window_mode, workspace=self.attn_ws)
         return self.o, self.lse

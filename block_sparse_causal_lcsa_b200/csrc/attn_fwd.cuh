@@ -87,6 +87,9 @@ struct AttnParams {
   int64_t osh, ost, osy, osx;  // strides of o (stream stride = H * osh)
   int32_t H, Tq, Y, X, Hb, Wb, nQT, nQB, kmax, cap;
   int32_t win, win_mode;     // token-level window (0: none), mode 2 truncate / 3 preserve
+  int32_t split_from;        // units >= split_from run as two CTAs over halves of their kept blocks
+  float* part_o;             // [split units][2][128][D] fp32 O of each half (normalised), or null
+  float* part_lse;           // [split units][2][128] natural-log LSE of each half
   float scale_log2;          // log2(e) / sqrt(D)
   uint64_t wait_limit_ns;
   unsigned int* err;
@@ -140,8 +143,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // CTA -> (stream*head, query block); within a head the query blocks of the
   // newest time step (the longest rows) go first.
   const int HbWb = p.Hb * p.Wb;
-  const int bh = blockIdx.x / p.nQB;
-  const int rr = blockIdx.x % p.nQB;
+  // CTA -> work unit. A grid whose last wave would be partly empty runs each of
+  // its last units as two CTAs over the two halves of the unit's kept blocks;
+  // attn_merge_kernel combines the halves.
+  int unit = blockIdx.x, half = -1;
+  if (static_cast<int>(blockIdx.x) >= p.split_from) {
+    const int k = blockIdx.x - p.split_from;
+    unit = p.split_from + (k >> 1);
+    half = k & 1;
+  }
+  const int bh = unit / p.nQB;
+  const int rr = unit % p.nQB;
   const int tq = p.nQT - 1 - rr / HbWb;
   const int sp = rr % HbWb;
   const int b = bh / p.H;
@@ -152,6 +164,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (n < 0 || n > p.kmax) {
     if (threadIdx.x == 0) atomicOr(p.err, DEVERR_BOUNDS);
     n = 0;
+  }
+  if (half >= 0) {
+    const int h0 = (n + 1) >> 1;
+    if (half == 0) {
+      n = h0;
+    } else {
+      blist += h0;
+      n -= h0;
+    }
   }
   const int64_t begin = p.kv_begin[b], end = p.kv_end[b];
   const int64_t m_first = begin >> 1;
@@ -190,7 +211,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // thread 0 is also the Q/K producer: it initialises the barriers and starts
     // the Q and first K copies right away, so their latency overlaps the
     // tensor-memory allocation and the CTA-wide barrier
-    const int first_blk = blist[0];              // row capacity kmax >= 1
+    const int first_blk = n > 0 ? blist[0] : 0;
     for (int i = 0; i < B_COUNT; ++i)
       mbar_init(bar(i), (i >= B_P_FULL && i < B_P_FULL + S_BUFS) ? SOFTMAX_THREADS : 1u);
     *abort_flag = 0;
@@ -437,7 +458,30 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int y = 8 * yq + yy, x = 8 * xq + xx;
     __nv_bfloat16* orow = p.o + static_cast<int64_t>(bh) * p.osh + static_cast<int64_t>(frame) * p.ost +
                           static_cast<int64_t>(y) * p.osy + static_cast<int64_t>(x) * p.osx;
-    if (done) {
+    if (half >= 0) {
+      // one half of a split unit: fp32 O (normalised) and LSE for the merge
+      const int64_t prow = (static_cast<int64_t>(unit - p.split_from) * 2 + half) * 128 + r;
+      float* po = p.part_o + prow * D;
+      if (done) tc_fence_after();
+      const float inv_l = done && l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        if (done) {
+          tmem_ld_32x32b_x32(t_lane + TMEM_O_COL + c0, o);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = 0u;
+        }
+#pragma unroll
+        for (int k = 0; k < 32; k += 4)
+          *reinterpret_cast<float4*>(po + c0 + k) =
+              make_float4(__uint_as_float(o[k]) * inv_l, __uint_as_float(o[k + 1]) * inv_l,
+                          __uint_as_float(o[k + 2]) * inv_l, __uint_as_float(o[k + 3]) * inv_l);
+      }
+      p.part_lse[prow] = done && l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+    } else if (done) {
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;   // a row with no visible key: O = 0
 #pragma unroll
@@ -471,6 +515,47 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// Combines the two halves of each split unit, one warp per query row:
+// O = (w0 O0 + w1 O1) / (w0 + w1) with w_h = exp(LSE_h - max), LSE = max + log(w0 + w1).
+template <int D>
+__global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__ AttnParams p, int32_t n_split) {
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= static_cast<int64_t>(n_split) * 128) return;
+  const int su = static_cast<int>(wid >> 7), r = static_cast<int>(wid & 127);
+  const int unit = p.split_from + su;
+  const int HbWb = p.Hb * p.Wb;
+  const int bh = unit / p.nQB, rr = unit % p.nQB;
+  const int tq = p.nQT - 1 - rr / HbWb, sp = rr % HbWb;
+  const int fq0 = p.Tq - 2 * p.nQT + 2 * tq;
+  if (fq0 < 0 && r < 64) return;                   // rows of a missing older frame
+  const int frame = fq0 + (r >> 6);
+  const int y = 8 * (sp / p.Wb) + ((r >> 3) & 7), x = 8 * (sp % p.Wb) + (r & 7);
+  const int64_t r0 = (static_cast<int64_t>(su) * 2) * 128 + r, r1 = r0 + 128;
+  const float l0 = p.part_lse[r0], l1 = p.part_lse[r1];
+  const float mx = fmaxf(l0, l1);
+  float w0 = 0.f, w1 = 0.f, lse = -INFINITY;
+  if (mx != -INFINITY) {
+    w0 = __expf(l0 - mx);
+    w1 = __expf(l1 - mx);
+    const float sum = w0 + w1;
+    lse = mx + __logf(sum);
+    w0 /= sum;
+    w1 /= sum;
+  }
+  __nv_bfloat16* orow = p.o + static_cast<int64_t>(bh) * p.osh + static_cast<int64_t>(frame) * p.ost +
+                        static_cast<int64_t>(y) * p.osy + static_cast<int64_t>(x) * p.osx;
+  const float* o0 = p.part_o + r0 * D;
+  const float* o1 = p.part_o + r1 * D;
+  for (int c = 2 * lane; c < D; c += 64) {
+    const float2 a = *reinterpret_cast<const float2*>(o0 + c);
+    const float2 b = *reinterpret_cast<const float2*>(o1 + c);
+    *reinterpret_cast<uint32_t*>(orow + c) = pack_bf16x2(w0 * a.x + w1 * b.x, w0 * a.y + w1 * b.y);
+  }
+  if (lane == 0 && p.lse != nullptr)
+    p.lse[((static_cast<int64_t>(bh) * p.Tq + frame) * p.Y + y) * p.X + x] = lse;
 }
 
 }  // namespace lcsa

@@ -38,6 +38,7 @@ uint64_t g_wait_limit_ns = kDefaultWaitNs;
 std::mutex g_mu;
 unsigned int* g_err_ptr[kMaxDevices] = {};
 bool g_attr_done[kMaxDevices] = {};
+int g_sm_count[kMaxDevices] = {};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -72,6 +73,9 @@ lcsa_status device_setup(int* dev_out, unsigned int** err_out) {
                              BwdLayout<128>::SMEM_KV) != cudaSuccess ||
         cudaFuncSetAttribute(bwd_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              BwdLayout<64>::SMEM_KV) != cudaSuccess)
+      return LCSA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        g_sm_count[dev] < 1)
       return LCSA_ERR_CUDA;
     g_attr_done[dev] = true;
   }
@@ -690,7 +694,8 @@ lcsa_status lcsa_select_blocks_noalloc(const double* q_pool, int32_t q_frames, c
 
 static lcsa_status attn_fwd_impl(const lcsa_tensor* q, const lcsa_kv_cache* kv, const int32_t* blk_idx,
                                  const int32_t* blk_cnt, int32_t kmax, int32_t window, int32_t window_mode,
-                                 lcsa_tensor* o, float* lse, lcsa_stream_t stream) {
+                                 lcsa_tensor* o, float* lse, void* workspace, size_t workspace_bytes,
+                                 lcsa_stream_t stream) {
   lcsa_status s = check_tensor(q);
   if (s != LCSA_OK) return s;
   if ((s = check_cache(kv)) != LCSA_OK) return s;
@@ -738,21 +743,39 @@ static lcsa_status attn_fwd_impl(const lcsa_tensor* q, const lcsa_kv_cache* kv, 
     p.kv_begin[b] = kv->begin[b] - base;
     p.kv_end[b] = kv->end[b] - base;
   }
-  const int64_t grid = static_cast<int64_t>(q->B) * q->H * p.nQB;  // one CTA per query block
-  if (grid > 0x7fffffff) return LCSA_ERR_SHAPE;
-  if (grid == 0) return LCSA_OK;
+  const int64_t units = static_cast<int64_t>(q->B) * q->H * p.nQB;  // one CTA per query block
+  if (units > 0x7fffffff / 2) return LCSA_ERR_SHAPE;
+  if (units == 0) return LCSA_OK;
+  // With a workspace, a last wave that would leave most SMs idle is evened
+  // out: its r units run as 2r half-units (the kept blocks split in two) and a
+  // merge kernel combines each pair.
+  const int64_t sms = g_sm_count[dev];
+  const int64_t r = units % sms;
+  int64_t grid = units;
+  p.split_from = 0x7fffffff;
+  if (workspace != nullptr && units > sms && r > 0 && 2 * r <= sms && r <= LCSA_ATTN_SPLIT_MAX &&
+      workspace_bytes >= static_cast<size_t>(2 * r * 128 * (q->D + 1) * 4) && aligned16(workspace)) {
+    p.split_from = static_cast<int32_t>(units - r);
+    p.part_o = static_cast<float*>(workspace);
+    p.part_lse = p.part_o + 2 * r * 128 * q->D;
+    grid = units + r;
+  }
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (q->D == 128)
     attn_fwd_kernel<128><<<static_cast<unsigned>(grid), ATTN_THREADS, AttnLayout<128>::SMEM_BYTES, cs>>>(tq, tk, tv, p);
   else
     attn_fwd_kernel<64><<<static_cast<unsigned>(grid), ATTN_THREADS, AttnLayout<64>::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+  if ((s = launched()) != LCSA_OK || grid == units) return s;
+  const unsigned mgrid = static_cast<unsigned>((r * 128 * 32 + 255) / 256);
+  if (q->D == 128) attn_merge_kernel<128><<<mgrid, 256, 0, cs>>>(p, static_cast<int32_t>(r));
+  else attn_merge_kernel<64><<<mgrid, 256, 0, cs>>>(p, static_cast<int32_t>(r));
   return launched();
 }
 
 lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_cache* kv, const int32_t* blk_idx,
                                  const int32_t* blk_cnt, int32_t kmax, lcsa_tensor* o, float* lse,
                                  lcsa_stream_t stream) {
-  return attn_fwd_impl(q, kv, blk_idx, blk_cnt, kmax, 0, LCSA_WINDOW_TRUNCATE_TOKENS, o, lse, stream);
+  return attn_fwd_impl(q, kv, blk_idx, blk_cnt, kmax, 0, LCSA_WINDOW_TRUNCATE_TOKENS, o, lse, nullptr, 0, stream);
 }
 
 lcsa_status lcsa_sparse_attn_fwd_window(const lcsa_tensor* q, const lcsa_kv_cache* kv, const int32_t* blk_idx,
@@ -761,7 +784,23 @@ lcsa_status lcsa_sparse_attn_fwd_window(const lcsa_tensor* q, const lcsa_kv_cach
   if (window < 0 || (window > 0 && window_mode != LCSA_WINDOW_TRUNCATE_TOKENS &&
                      window_mode != LCSA_WINDOW_PRESERVE_TOKENS))
     return LCSA_ERR_INVALID_ARG;
-  return attn_fwd_impl(q, kv, blk_idx, blk_cnt, kmax, window, window_mode, o, lse, stream);
+  return attn_fwd_impl(q, kv, blk_idx, blk_cnt, kmax, window, window_mode, o, lse, nullptr, 0, stream);
+}
+
+size_t lcsa_sparse_attn_fwd_workspace_bytes(int32_t head_dim) {
+  if (head_dim != 64 && head_dim != 128) return 0;
+  return static_cast<size_t>(2) * LCSA_ATTN_SPLIT_MAX * 128 * (head_dim + 1) * 4;
+}
+
+lcsa_status lcsa_sparse_attn_fwd_ex(const lcsa_tensor* q, const lcsa_kv_cache* kv, const int32_t* blk_idx,
+                                    const int32_t* blk_cnt, int32_t kmax, int32_t window, int32_t window_mode,
+                                    lcsa_tensor* o, float* lse, void* workspace, size_t workspace_bytes,
+                                    lcsa_stream_t stream) {
+  if (window < 0 || (window > 0 && window_mode != LCSA_WINDOW_TRUNCATE_TOKENS &&
+                     window_mode != LCSA_WINDOW_PRESERVE_TOKENS))
+    return LCSA_ERR_INVALID_ARG;
+  return attn_fwd_impl(q, kv, blk_idx, blk_cnt, kmax, window, window > 0 ? window_mode : LCSA_WINDOW_TRUNCATE_TOKENS,
+                       o, lse, workspace, workspace_bytes, stream);
 }
 
 lcsa_status lcsa_last_device_error(lcsa_stream_t stream) {

@@ -332,6 +332,25 @@ LCSA_API lcsa_status lcsa_sparse_attn_fwd_window(const lcsa_tensor* q, const lcs
                                         lcsa_tensor* o, float* lse, lcsa_stream_t stream);
 
 /*
+ * lcsa_sparse_attn_fwd_ex - lcsa_sparse_attn_fwd_window with an optional
+ * workspace (device, 16-byte aligned, owned by the caller) of
+ * lcsa_sparse_attn_fwd_workspace_bytes(D) bytes. With it, when the query
+ * blocks do not fill the GPU's last wave of CTAs (one CTA per SM) and at most
+ * half the SMs would be busy in it, each of those last query blocks runs as
+ * two CTAs over the two halves of its kept blocks and a second kernel merges
+ * the halves (fp32, by their log-sum-exps); without it (NULL) the result is
+ * computed as by lcsa_sparse_attn_fwd. Both give the same output up to fp32
+ * rounding of the merge. At most LCSA_ATTN_SPLIT_MAX query blocks are split.
+ */
+#define LCSA_ATTN_SPLIT_MAX 128
+LCSA_API size_t lcsa_sparse_attn_fwd_workspace_bytes(int32_t head_dim);
+LCSA_API lcsa_status lcsa_sparse_attn_fwd_ex(const lcsa_tensor* q, const lcsa_kv_cache* kv,
+                                    const int32_t* blk_idx, const int32_t* blk_cnt,
+                                    int32_t kmax, int32_t window, int32_t window_mode,
+                                    lcsa_tensor* o, float* lse, void* workspace,
+                                    size_t workspace_bytes, lcsa_stream_t stream);
+
+/*
  * lcsa_segment_blocks - block lists for dense attention confined to one
  * segment (section 2.2, stage 1: joint video-image training with a
  * block-diagonal segment mask, so that attention stays inside one video clip
