@@ -5,8 +5,8 @@
 //
 // Two kernels, joined by a caller-provided workspace of 64-bit keys
 // [rows][c_stride]:
-// score_kernel  one CTA per (8 query blocks) x (64 candidate key blocks) of a
-//   (stream, head, temporal block). The 8 pooled query rows and the 64 pooled
+// score_kernel  one CTA per (16 query blocks) x (32 candidate key blocks) of a
+//   (stream, head, temporal block). The 16 pooled query rows and the 32 pooled
 //   key rows are staged in shared memory (key rows padded to D+1 doubles so
 //   the 32 lanes of a warp, each reading its own row, hit distinct banks);
 //   each thread scores one candidate against 4 rows - 4 independent float64
@@ -26,9 +26,9 @@
 
 namespace lcsa {
 
-constexpr int SC_ROWS = 8;        // query blocks per score CTA
-constexpr int SC_CANDS = 64;      // candidate key blocks per score CTA
-constexpr int SC_THREADS = 128;   // 64 candidates x 2 groups of 4 rows
+constexpr int SC_ROWS = 16;       // query blocks per score CTA
+constexpr int SC_CANDS = 32;      // candidate key blocks per score CTA
+constexpr int SC_THREADS = 128;   // 32 candidates x 4 groups of 4 rows
 
 struct SelectParams {
   const double* q_pool;   // [B][H][nQT][Hb][Wb][D]
@@ -153,7 +153,7 @@ score_kernel(const __grid_constant__ SelectParams p) {
   constexpr int V2 = D / 2;                       // 16-byte vectors per pooled row
   constexpr int PER_LANE = V2 / 32;               // vectors per lane per row
   constexpr int ROWS_PER_WARP = SC_CANDS / (SC_THREADS / 32);
-  // query rows: warp w stages rows w, w+4 (plain copy, zero beyond nrows)
+  // query rows: warp w stages rows w, w+4, ... (plain copy, zero beyond nrows)
   const double2* qsrc = reinterpret_cast<const double2*>(
       p.q_pool + (static_cast<int64_t>(bh) * nQB + tq * HbWb + sp0) * D);
 #pragma unroll
@@ -166,7 +166,7 @@ score_kernel(const __grid_constant__ SelectParams p) {
       qs[rr * D + 2 * e + 1] = x.y;
     }
   }
-  // candidate rows: warp w stages rows w*16 .. w*16+15, all loads issued before
+  // candidate rows: warp w stages ROWS_PER_WARP consecutive rows, all loads issued before
   // any store so that the L2 round trips overlap
   double2 buf[ROWS_PER_WARP][PER_LANE];
 #pragma unroll
