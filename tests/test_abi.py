@@ -110,3 +110,76 @@ def test_select_kmax_host_rule(lib):
     assert lib.lcsa_select_kmax(C.byref(kv), 2, C.byref(sp)) == 34  # 243 candidates
     # workspace: 12 heads x 252 query blocks x 756 causal candidates x 8 bytes
     assert lib.lcsa_select_workspace_bytes(C.byref(kv), 2) == 12 * 252 * 756 * 8
+
+
+def test_kv_advance_host_state(lib):
+    """lcsa_kv_advance applies an append's cache-state update with no device
+    work: first odd chunk, steady appends, eviction at the capacity."""
+    from block_sparse_causal_lcsa_b200 import _abi
+    kv = _abi.KVCacheStruct()
+    kv.k, kv.v, kv.k_pool = 0x1000, 0x2000, 0x3000
+    kv.B, kv.H, kv.cap_frames, kv.Y, kv.X, kv.D = 2, 1, 6, 16, 16, 128
+    assert lib.lcsa_kv_advance(C.byref(kv), 3, 1, 0) == _abi.OK          # odd first chunk of stream 0
+    assert (kv.begin[0], kv.end[0]) == (1, 4)
+    assert lib.lcsa_kv_advance(C.byref(kv), 1, 1, 0) == _abi.ERR_SHAPE   # odd chunk on a non-empty stream
+    for _ in range(3):
+        assert lib.lcsa_kv_advance(C.byref(kv), 2, 2, 0) == _abi.OK
+    assert (kv.begin[0], kv.end[0]) == (4, 10)                           # the newest 6 frames
+    assert (kv.begin[1], kv.end[1]) == (0, 6)
+    assert lib.lcsa_kv_advance(C.byref(kv), 2, 2, 1) == _abi.ERR_INVALID_ARG   # streams 1..2 of 2
+    assert lib.lcsa_kv_advance(None, 2, 1, 0) == _abi.ERR_INVALID_ARG
+
+
+def test_new_entry_points_reject_bad_arguments(lib):
+    from block_sparse_causal_lcsa_b200 import _abi
+    kv = _abi.KVCacheStruct()
+    kv.k, kv.v, kv.k_pool = 0x1000, 0x2000, 0x3000
+    kv.B, kv.H, kv.cap_frames, kv.Y, kv.X, kv.D = 1, 1, 6, 16, 16, 128
+    kv.begin[0], kv.end[0] = 0, 6
+    t = _abi.Tensor(0x1000, 1, 1, 2, 16, 16, 128, 65536, 65536, 32768, 2048, 128)
+    # token-window attention needs a token-level mode
+    assert lib.lcsa_sparse_attn_fwd_window(C.byref(t), C.byref(kv), 0x5000, 0x6000, 4, 72, 0, C.byref(t), None,
+                                           None) == _abi.ERR_INVALID_ARG
+    assert lib.lcsa_sparse_attn_fwd_ex(C.byref(t), C.byref(kv), 0x5000, 0x6000, 4, -1, 2, C.byref(t), None, None, 0,
+                                       None) == _abi.ERR_INVALID_ARG
+    # window modes: token windows may be even, block windows may not; unknown modes are rejected
+    sp = _abi.SelectParamsStruct(0, 72, 2, 64, 0.136, 1e-5)
+    ws = lib.lcsa_select_workspace_bytes(C.byref(kv), 2)
+    sp.window_mode = 4
+    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, 0x7000, ws, None) == \
+        _abi.ERR_INVALID_ARG
+    sp.window_mode = 1
+    assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, 0x7000, ws, None) == \
+        _abi.ERR_INVALID_ARG
+    # segment lists: capacity below the longest segment's key blocks, segments longer than the queries
+    assert lib.lcsa_segment_kmax(C.byref(kv)) == 3 * 4
+    assert lib.lcsa_segment_blocks(6, C.byref(kv), 11, 0x5000, 0x6000, None) == _abi.ERR_CAPACITY
+    assert lib.lcsa_segment_blocks(4, C.byref(kv), 12, 0x5000, 0x6000, None) == _abi.ERR_SHAPE
+    # backward: workspace too small
+    need = lib.lcsa_sparse_attn_bwd_workspace_bytes(C.byref(kv), 2)
+    assert need > 0
+    assert lib.lcsa_sparse_attn_bwd(C.byref(t), C.byref(kv), 0x5000, 0x6000, 4, C.byref(t), 0x8000, C.byref(t),
+                                    C.byref(t), 0x9000, 0xA000, 0xB000, need - 16, None) == _abi.ERR_WORKSPACE
+    assert lib.lcsa_sparse_attn_fwd_workspace_bytes(128) == 2 * 128 * 128 * 129 * 4
+    assert lib.lcsa_sparse_attn_fwd_workspace_bytes(96) == 0
+
+
+@pytest.mark.parametrize("mode,window", [(2, 72), (3, 72), (2, 20), (3, 35), (0, 9), (1, 9)])
+def test_select_kmax_covers_every_row(lib, mode, window):
+    """The host capacity rule bounds K_i of every row, token windows included
+    (checked against the oracle's window and K rules)."""
+    from block_sparse_causal_lcsa_b200 import _abi
+    from oracle import lcsa_oracle as orc
+    kv = _abi.KVCacheStruct()
+    kv.B, kv.H, kv.cap_frames, kv.Y, kv.X, kv.D = 1, 1, 6, 96, 168, 128
+    kv.begin[0], kv.end[0] = 0, 6
+    sp = _abi.SelectParamsStruct(0, window, mode, 0, 0.136, 1e-5)
+    kmax = lib.lcsa_select_kmax(C.byref(kv), 2, C.byref(sp))
+    Hb, Wb = 12, 21
+    Ks = []
+    for i in range(Hb * Wb):
+        yq, xq = divmod(i, Wb)
+        C_i = int(orc.allowed_blocks(2, yq, xq, 3, Hb, Wb, window, mode).sum())
+        Ks.append(orc.top_k_count(C_i, 0, 0.136))
+    assert kmax >= max(Ks)
+    assert kmax <= max(Ks) + 1 or mode >= 2
