@@ -432,12 +432,13 @@ def run_ours(args, world, rank, local):
         if rec.get("source_hash", "").strip() == attn_source_hash():
             traffic = int(rec["bytes_per_launch"])
 
-    # kernels per step: pool, the fused append (streaming), score + top-K, the
+    # kernels per timed step: the ingest (streaming graph: Q pooling and the
+    # fused K/V append in one launch; clip: Q and K pooling), score + top-K, the
     # attention and, when its last wave is split, the merge of the halves
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     units = w.B * w.H * ((w.q_frames + 1) // 2) * w.Hb * w.Wb
     split = units > sms and 0 < units % sms <= sms // 2
-    launches_per_step = (2 if streaming else 1) + 2 + (2 if split else 1)
+    launches_per_step = 1 + 2 + (2 if split else 1)
     # the headline is the step as a user runs it in production: replayed from a
     # CUDA graph (same kernels, same work, one launch); the eager run with CUDA
     # events between the kernels gives the per-kernel split

@@ -18,6 +18,7 @@ from .api import (  # noqa: F401
     debug_exp2_poly,
     debug_set_wait_limit_ns,
     debug_stalled_wait,
+    ingest_chunk,
     kv_append,
     last_device_error,
     pool_qk,

@@ -66,6 +66,8 @@ PROTOTYPES = {
                                C.c_void_p]),
     "lcsa_kv_append": (C.c_int, [C.POINTER(KVCacheStruct), C.POINTER(Tensor), C.POINTER(Tensor),
                                  C.c_void_p, C.c_int32, C.c_void_p]),
+    "lcsa_ingest_chunk": (C.c_int, [C.POINTER(Tensor), C.c_void_p, C.POINTER(KVCacheStruct), C.POINTER(Tensor),
+                                    C.POINTER(Tensor), C.c_int32, C.c_void_p]),
     "lcsa_kv_advance": (C.c_int, [C.POINTER(KVCacheStruct), C.c_int32, C.c_int32, C.c_int32]),
     "lcsa_select_kmax": (C.c_int32, [C.POINTER(KVCacheStruct), C.c_int32,
                                      C.POINTER(SelectParamsStruct)]),

@@ -147,6 +147,19 @@ def kv_append(cache: KVCache, k_new: torch.Tensor, v_new: torch.Tensor,
            "lcsa_kv_append")
 
 
+def ingest_chunk(q: torch.Tensor, cache: KVCache, k_new: torch.Tensor, v_new: torch.Tensor,
+                 q_pool: Optional[torch.Tensor] = None, stream_offset: int = 0,
+                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """pool_qk(q) and kv_append(cache, k_new, v_new) (K pooled on the way) in
+    one launch; returns q_pool."""
+    if q_pool is None:
+        q_pool = torch.empty(pooled_shape(q), dtype=torch.float64, device=q.device)
+    qd, kd, vd = tensor_desc(q), tensor_desc(k_new), tensor_desc(v_new)
+    _check(_lib.lcsa_ingest_chunk(C.byref(qd), q_pool.data_ptr(), C.byref(cache.struct), C.byref(kd), C.byref(vd),
+                                  stream_offset, _stream(stream)), "lcsa_ingest_chunk")
+    return q_pool
+
+
 @dataclass
 class SelectParams:
     top_k: int = 0
@@ -405,8 +418,7 @@ class StreamingStep:
 
     def __call__(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
                  stream: Optional[torch.cuda.Stream] = None):
-        pool_qk(q, None, self.q_pool, None, stream)
-        kv_append(self.cache, k_new, v_new, None, 0, stream)
+        ingest_chunk(q, self.cache, k_new, v_new, self.q_pool, 0, stream)
         select_blocks(self.q_pool, self.q_frames, self.cache, self.params, self.kmax,
                       self.blk_idx, self.blk_cnt, self.workspace, stream)
         tw = self.params.window if self.params.window_mode >= WINDOW_TRUNCATE_TOKENS else 0

@@ -298,8 +298,11 @@ lcsa_status lcsa_pool_qk(const lcsa_tensor* q, const lcsa_tensor* k, double* q_p
   return launch_ingest(p, q->D, static_cast<cudaStream_t>(stream));
 }
 
-lcsa_status lcsa_kv_append(lcsa_kv_cache* kv, const lcsa_tensor* k_new, const lcsa_tensor* v_new,
-                           const double* k_pool_new, int32_t stream_offset, lcsa_stream_t stream) {
+// lcsa_kv_append, optionally with the pooling of q into q_pool in the same
+// launch (only on the fused path, where K is pooled while it is copied).
+static lcsa_status kv_append_impl(lcsa_kv_cache* kv, const lcsa_tensor* k_new, const lcsa_tensor* v_new,
+                                  const double* k_pool_new, int32_t stream_offset, lcsa_stream_t stream,
+                                  const lcsa_tensor* q, double* q_pool) {
   lcsa_status s = check_cache(kv);
   if (s != LCSA_OK) return s;
   if ((s = check_tensor(k_new)) != LCSA_OK || (s = check_tensor(v_new)) != LCSA_OK) return s;
@@ -344,6 +347,13 @@ lcsa_status lcsa_kv_append(lcsa_kv_cache* kv, const lcsa_tensor* k_new, const lc
     }
     ip.t[0].pool_out = kv->k_pool;
     ip.t[0].pool_ring = 1;
+    if (q != nullptr) {
+      IngestTensor& it = ip.t[2];
+      set_ingest_source(it, q);
+      it.tb_first = 0;
+      it.units = static_cast<int64_t>(q->B) * q->H * it.nT * ip.Hb * ip.Wb;
+      it.pool_out = q_pool;
+    }
     if ((s = launch_ingest(ip, kn->D, static_cast<cudaStream_t>(stream))) != LCSA_OK) return s;
     for (int bn = 0; bn < kn->B; ++bn) {
       kv->begin[bn + stream_offset] = new_begin[bn];
@@ -382,6 +392,22 @@ lcsa_status lcsa_kv_append(lcsa_kv_cache* kv, const lcsa_tensor* k_new, const lc
     kv->end[bn + stream_offset] = new_end[bn];
   }
   return LCSA_OK;
+}
+
+lcsa_status lcsa_kv_append(lcsa_kv_cache* kv, const lcsa_tensor* k_new, const lcsa_tensor* v_new,
+                           const double* k_pool_new, int32_t stream_offset, lcsa_stream_t stream) {
+  return kv_append_impl(kv, k_new, v_new, k_pool_new, stream_offset, stream, nullptr, nullptr);
+}
+
+lcsa_status lcsa_ingest_chunk(const lcsa_tensor* q, double* q_pool, lcsa_kv_cache* kv, const lcsa_tensor* k_new,
+                              const lcsa_tensor* v_new, int32_t stream_offset, lcsa_stream_t stream) {
+  lcsa_status s = check_tensor(q);
+  if (s != LCSA_OK) return s;
+  if (kv == nullptr) return LCSA_ERR_INVALID_ARG;
+  if (q_pool == nullptr) return LCSA_ERR_INVALID_ARG;
+  if (!aligned16(q_pool)) return LCSA_ERR_ALIGN;
+  if (q->H != kv->H || q->Y != kv->Y || q->X != kv->X || q->D != kv->D) return LCSA_ERR_SHAPE;
+  return kv_append_impl(kv, k_new, v_new, nullptr, stream_offset, stream, q, q_pool);
 }
 
 lcsa_status lcsa_kv_advance(lcsa_kv_cache* kv, int32_t frames, int32_t n_streams, int32_t stream_offset) {

@@ -193,6 +193,17 @@ LCSA_API lcsa_status lcsa_kv_append(lcsa_kv_cache* kv, const lcsa_tensor* k_new,
                            int32_t stream_offset, lcsa_stream_t stream);
 
 /*
+ * lcsa_ingest_chunk - lcsa_pool_qk of the queries and lcsa_kv_append of the
+ * chunk's keys and values (K pooled on the way) in one launch: q is pooled
+ * into q_pool (layout as lcsa_pool_qk's q_pool), k_new / v_new are written
+ * into the cache as by lcsa_kv_append with k_pool_new = NULL. Same errors as
+ * those two calls; q's H, Y, X, D must match the cache.
+ */
+LCSA_API lcsa_status lcsa_ingest_chunk(const lcsa_tensor* q, double* q_pool, lcsa_kv_cache* kv,
+                              const lcsa_tensor* k_new, const lcsa_tensor* v_new,
+                              int32_t stream_offset, lcsa_stream_t stream);
+
+/*
  * lcsa_kv_advance - the host-side part of lcsa_kv_append alone: advance the
  * begin / end of streams [stream_offset, stream_offset + n_streams) as
  * appending `frames` frames would, launching nothing. For replaying a

@@ -190,6 +190,27 @@ def test_tail_split_matches_unsplit_and_oracle(lc):
     compare_all(w, x, g, heads=[0, 5, 11])
 
 
+def test_ingest_chunk_equals_pool_then_append(lc):
+    """One launch for Q pooling and the fused K/V append gives the same q_pool
+    and cache as pool_qk followed by kv_append, bit for bit (two streams, an
+    odd first chunk, then a wrapped ring)."""
+    H, Y, X, D, cap = 2, 16, 24, 128, 4
+    a = lc.KVCache(2, H, cap, Y, X, D)
+    b = lc.KVCache(2, H, cap, Y, X, D)
+    for c in (a, b):
+        c.k.zero_(), c.v.zero_(), c.k_pool.zero_()
+    g = torch.Generator().manual_seed(17)
+    for t in (3, 2, 2, 2):
+        q, k, v = (torch.randn((2, H, t, Y, X, D), generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+        qp_a = lc.ingest_chunk(q, a, k, v)
+        qp_b = lc.pool_qk(q)[0]
+        lc.kv_append(b, k, v)
+        torch.cuda.synchronize()
+        assert torch.equal(qp_a, qp_b) and a.state() == b.state()
+    assert lc.last_device_error() == 0
+    assert torch.equal(a.k, b.k) and torch.equal(a.v, b.v) and torch.equal(a.k_pool, b.k_pool)
+
+
 def test_graph_replay_equals_eager_steps(lc):
     """Eight 2-frame chunks through a 6-frame cache, eagerly and from CUDA graphs
     (one per ring phase): identical outputs, cache contents and state."""
