@@ -220,6 +220,7 @@ def run_ours(args, world, rank, local):
                                 for _ in range(3)))
         step = lc.StreamingStep(cache, w.q_frames, params)
         base_state = cache.state()
+        tok_window = w.window if w.window_mode >= li.WINDOW_TRUNCATE_TOKENS else 0
 
         def run_step(i, q=None, k=None, v=None, ev=None):
             if q is None:
@@ -239,7 +240,8 @@ def run_ours(args, world, rank, local):
                              step.blk_idx, step.blk_cnt, step.workspace)
             if ev is not None:
                 ev[3].record()
-            lc.sparse_attn_fwd(q, step.cache, step.blk_idx, step.blk_cnt, step.o, step.lse, workspace=step.attn_ws)
+            lc.sparse_attn_fwd(q, step.cache, step.blk_idx, step.blk_cnt, step.o, step.lse, workspace=step.attn_ws,
+                               window=tok_window, window_mode=w.window_mode)
             if ev is not None:
                 ev[4].record()
             return step.o

@@ -381,9 +381,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const uint32_t ym = ((1u << yhi) - 1u) & ~((1u << ylo) - 1u);
         const uint32_t xm = ((1u << xhi) - 1u) & ~((1u << xlo) - 1u);
         if (ym != 0xFFu || xm != 0xFFu) {
+          // 64-bit visibility of the frame's 8 x 8 tokens (bit 8*yy + xx): the
+          // x mask in every byte, kept for the rows in the window; the block's
+          // two frames share it
+          const uint64_t xrep = static_cast<uint64_t>(xm) * 0x0101010101010101ull;
+          const uint64_t yhi_m = yhi >= 8 ? ~0ull : (1ull << (8 * yhi)) - 1ull;
+          const uint64_t ylo_m = ylo >= 8 ? ~0ull : (1ull << (8 * ylo)) - 1ull;
+          const uint64_t vis = xrep & yhi_m & ~ylo_m;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (!((ym >> ((c >> 3) & 7)) & (xm >> (c & 7)) & 1u)) s[c] = __float_as_uint(-INFINITY);
+          for (int c = 0; c < 64; ++c) {
+            if (!((vis >> c) & 1ull)) {
+              s[c] = __float_as_uint(-INFINITY);
+              s[c + 64] = __float_as_uint(-INFINITY);
+            }
+          }
         }
       }
       float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;

@@ -352,4 +352,119 @@ topk_kernel(const __grid_constant__ SelectParams p) {
   if (tid == 0) p.blk_cnt[row] = K;
 }
 
+// One warp per query block (4 per CTA), for launches with many rows: the
+// row's keys sit in registers (candidate j = 32*i + lane in slot i, at most
+// 32*KPL candidates) and each radix pass is one ballot per slot, with no
+// CTA-wide barrier; the same selection as topk_kernel.
+constexpr int TKW_WARPS = 4;
+template <int KPL>
+__global__ void __launch_bounds__(TKW_WARPS * 32)
+topk_warp_kernel(const __grid_constant__ SelectParams p) {
+  const int HbWb = p.Hb * p.Wb;
+  const int nQB = p.nQT * HbWb;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * TKW_WARPS + warp;
+  if (row >= static_cast<int64_t>(p.B) * p.H * nQB) return;
+  const int bh = static_cast<int>(row / nQB);
+  const int qi = static_cast<int>(row % nQB);
+  const int tq = qi / HbWb, sp = qi % HbWb;
+  const StreamGeom g = stream_geom(p, bh / p.H, tq);
+  const int ncand = g.ncand;
+  if (ncand > 32 * KPL) {
+    if (lane == 0) atomicOr(p.err, DEVERR_BOUNDS);
+    return;
+  }
+  int y0, y1, x0, x1;
+  window_bounds(sp / p.Wb, p.Hb, p.window, p.window_mode, y0, y1);
+  window_bounds(sp % p.Wb, p.Wb, p.window, p.window_mode, x0, x1);
+  const int C = (g.tq_kv + 1) * (y1 - y0) * (x1 - x0);
+  int K;
+  if (p.top_k > 0) {
+    K = min(C, p.top_k);
+  } else {
+    const double kd = ceil(__dmul_rn(p.density, static_cast<double>(C)));
+    K = min(C, max(1, static_cast<int>(kd)));
+  }
+  const uint64_t* krow = p.keys + row * p.c_stride;
+  const int nslots = (ncand + 31) / 32;
+  uint64_t key[KPL];
+  bool act[KPL];
+  int nact = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    const int j = 32 * i + lane;
+    key[i] = (i < nslots && j < ncand) ? krow[j] : 0ull;
+    act[i] = key[i] != 0ull;                   // window-masked candidates are not ranked
+    if (i < nslots) nact += __popc(__ballot_sync(0xffffffffu, act[i]));
+  }
+  // exact K-th largest key, one bit at a time from the top (as topk_kernel)
+  uint64_t prefix = 0;
+  int krem = K;
+  int bit = 63;
+  for (; bit >= 0 && nact > 1; --bit) {
+    int cnt = 0;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+      if (i >= nslots) break;
+      cnt += __popc(__ballot_sync(0xffffffffu, act[i] && ((key[i] >> bit) & 1ull)));
+    }
+    const uint64_t chosen = cnt >= krem ? 1ull : 0ull;
+    if (chosen) {
+      nact = cnt;
+    } else {
+      krem -= cnt;
+      nact -= cnt;
+    }
+    prefix |= chosen << bit;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) act[i] = act[i] && ((key[i] >> bit) & 1ull) == chosen;
+  }
+  if (bit >= 0) {  // a single key matches the prefix: it is the K-th largest
+    uint64_t found = 0ull;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+      if (i >= nslots) break;
+      const uint32_t m = __ballot_sync(0xffffffffu, act[i]);
+      if (m) {
+        const int src = __ffs(m) - 1;
+        found = (static_cast<uint64_t>(__shfl_sync(0xffffffffu, static_cast<uint32_t>(key[i] >> 32), src)) << 32) |
+                __shfl_sync(0xffffffffu, static_cast<uint32_t>(key[i]), src);
+      }
+    }
+    prefix = found;
+  }
+  const double tau = key_value(prefix);
+  const uint64_t k_hi = order_key(__dadd_rn(tau, p.tie_eps));
+  const uint64_t k_lo = order_key(__dsub_rn(tau, p.tie_eps));
+  int above = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    if (i >= nslots) break;
+    above += __popc(__ballot_sync(0xffffffffu, key[i] > k_hi));
+  }
+  const int need = K - above;
+  int32_t* out = p.blk_idx + row * p.kmax;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int n_band = 0, n_sel = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    if (i >= nslots) break;
+    const int j = 32 * i + lane;
+    const bool in_above = key[i] > k_hi;
+    const bool in_band = key[i] >= k_lo && key[i] <= k_hi;
+    const uint32_t band_mask = __ballot_sync(0xffffffffu, in_band);
+    const bool take = in_above || (in_band && (n_band + __popc(band_mask & lt_mask)) < need);
+    const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int pos = n_sel + __popc(take_mask & lt_mask);
+      if (pos < p.kmax) out[pos] = j;
+      else atomicOr(p.err, DEVERR_BOUNDS);
+    }
+    n_band += __popc(band_mask);
+    n_sel += __popc(take_mask);
+  }
+  for (int pos = K + lane; pos < p.kmax; pos += 32) out[pos] = -1;
+  if (lane == 0) p.blk_cnt[row] = K;
+}
+
 }  // namespace lcsa
