@@ -341,30 +341,31 @@ def run_ours(args, world, rank, local):
     # the output read back, copies inside the timed region
     e2e = None
     if streaming:
+        # chunks from pinned host memory through lc.HostPipeline: each chunk's
+        # inputs cross PCIe while the previous chunk computes, and its O comes
+        # back on a third stream; the timed region runs from the first timed
+        # chunk's host-to-device copy to the last chunk's device-to-host copy
         hq = chunks[0][0].cpu().pin_memory()
         hk = chunks[0][1].cpu().pin_memory()
         hv = chunks[0][2].cpu().pin_memory()
         ho = torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory()
-        dq, dk, dv = torch.empty_like(chunks[0][0]), torch.empty_like(chunks[0][1]), torch.empty_like(chunks[0][2])
-        e_start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        e_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        pipe = lc.HostPipeline(step)
+        e_start = torch.cuda.Event(enable_timing=True)
+        done = None
         for i in range(args.warmup + args.steps):
+            if i == args.warmup:
+                torch.cuda.synchronize()
+                e_start.record(pipe.h2d_stream)
             flush_l2()
-            if i >= args.warmup:
-                e_start[i - args.warmup].record()
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            out = run_step(i, dq, dk, dv)
-            ho.copy_(out, non_blocking=True)
-            if i >= args.warmup:
-                e_end[i - args.warmup].record()
+            step.cache.set_state(base_state)
+            done = pipe.submit(hq, hk, hv, ho)
         torch.cuda.synchronize()
-        e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(e_start, e_end))
+        e2e_ms = e_start.elapsed_time(done) / args.steps
         e2e_ms = max_over_ranks(e2e_ms, world)
         e2e = {"value": whole_job_ms_per_chunk(e2e_ms, chunks_per_step, world), "unit": UNIT,
                "h2d_bytes_per_step": hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2,
-               "d2h_bytes_per_step": ho.numel() * 2}
+               "d2h_bytes_per_step": ho.numel() * 2,
+               "pipelined": "copies of chunk i+1 overlap the compute of chunk i (lc.HostPipeline)"}
     else:
         hq = q.cpu().pin_memory()
         hk = k.cpu().pin_memory()

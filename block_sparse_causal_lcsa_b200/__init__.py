@@ -6,6 +6,7 @@ selection (causal + locality window + top-K), tcgen05 sparse attention and
 the streaming KV-cache append.
 """
 from .api import (  # noqa: F401
+    HostPipeline,
     KVCache,
     LcsaError,
     SelectParams,

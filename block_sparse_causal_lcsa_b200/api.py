@@ -425,3 +425,68 @@ class StreamingStep:
         sparse_attn_fwd(q, self.cache, self.blk_idx, self.blk_cnt, self.o, self.lse, stream=stream,
                         window=tw, window_mode=self.params.window_mode, workspace=self.attn_ws)
         return self.o, self.lse
+
+
+class HostPipeline:
+    """Streams chunks from pinned host memory through a StreamingStep, with the
+    copies of one chunk overlapping the compute of its neighbours (a streaming
+    video stage receives frames from the host and returns them there).
+
+    Host-to-device copies run on their own stream into two alternating device
+    input sets; the step runs on the caller's current stream once its inputs
+    have landed; the device-to-host copy of O runs on a third stream. Inputs
+    of chunk i+1 therefore cross PCIe while chunk i computes and chunk i-1's
+    output travels back. All ordering is by CUDA events; nothing blocks the
+    host. `submit` returns the event that completes when O is in `ho`.
+    """
+
+    def __init__(self, step: StreamingStep):
+        self.step = step
+        self.h2d_stream = torch.cuda.Stream(device=step.o.device)
+        self.d2h_stream = torch.cuda.Stream(device=step.o.device)
+        self._bufs = None
+        self._in_ready = [torch.cuda.Event(), torch.cuda.Event()]
+        self._in_free = [None, None]
+        self._out_free = None
+        self._n = 0
+
+    def submit(self, hq: torch.Tensor, hk: torch.Tensor, hv: torch.Tensor,
+               ho: torch.Tensor) -> torch.cuda.Event:
+        for t in (hq, hk, hv, ho):
+            if t.is_cuda or not t.is_pinned():
+                raise ValueError("HostPipeline takes pinned host tensors")
+        if ho.shape != self.step.o.shape or ho.dtype != self.step.o.dtype:
+            raise ValueError("ho must match the step's output %s %s" % (tuple(self.step.o.shape), self.step.o.dtype))
+        dev = self.step.o.device
+        if self._bufs is None:
+            self._bufs = [tuple(torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (hq, hk, hv))
+                          for _ in range(2)]
+        slot = self._n & 1
+        dq, dk, dv = self._bufs[slot]
+        if dq.shape != hq.shape or dk.shape != hk.shape or dv.shape != hv.shape:
+            raise ValueError("chunk shapes must stay the same across submits")
+        # inputs: wait until the step that last read this slot has finished
+        if self._in_free[slot] is not None:
+            self.h2d_stream.wait_event(self._in_free[slot])
+        with torch.cuda.stream(self.h2d_stream):
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            self._in_ready[slot].record(self.h2d_stream)
+        cur = torch.cuda.current_stream(dev)
+        cur.wait_event(self._in_ready[slot])
+        # O is overwritten by this step: the previous read-back must be done
+        if self._out_free is not None:
+            cur.wait_event(self._out_free)
+        o, _ = self.step(dq, dk, dv)
+        computed = torch.cuda.Event()
+        computed.record(cur)
+        self._in_free[slot] = computed
+        self.d2h_stream.wait_event(computed)
+        done = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.d2h_stream):
+            ho.copy_(o, non_blocking=True)
+            done.record(self.d2h_stream)
+        self._out_free = done
+        self._n += 1
+        return done

@@ -236,6 +236,49 @@ def test_graph_replay_equals_eager_steps(lc):
     assert len(steps[1]._graphs) == 6
 
 
+def test_host_pipeline_equals_eager_steps(lc):
+    """Six chunks from pinned host memory through HostPipeline (copies on their
+    own streams, two alternating input sets) against the same chunks stepped
+    eagerly from device memory: identical outputs and cache contents."""
+    w = li.Workload("hostpipe", B=1, H=2, D=128, Y=16, X=24, q_frames=2, kv_past=(0,), cap_frames=6,
+                    density=0.4, seed=93)
+    caches = [lc.KVCache(w.B, w.H, w.cap_frames, w.Y, w.X, w.D) for _ in range(2)]
+    for c in caches:
+        c.k.zero_(), c.v.zero_(), c.k_pool.zero_()
+    steps = [lc.StreamingStep(c, 2, params_of(lc, w)) for c in caches]
+    pipe = lc.HostPipeline(steps[1])
+    g = torch.Generator().manual_seed(8)
+    shp = (w.B, w.H, 2, w.Y, w.X, w.D)
+    chunks = [tuple(torch.randn(shp, generator=g).to(torch.bfloat16).pin_memory() for _ in range(3))
+              for _ in range(6)]
+    outs = [torch.empty(shp, dtype=torch.bfloat16).pin_memory() for _ in range(6)]
+    done = [pipe.submit(*c, outs[t]) for t, c in enumerate(chunks)]
+    ref = []
+    for c in chunks:
+        o, _ = steps[0](*(t.cuda() for t in c))
+        ref.append(o.cpu())
+    done[-1].synchronize()
+    torch.cuda.synchronize()
+    assert lc.last_device_error() == 0
+    for t in range(6):
+        assert torch.equal(outs[t], ref[t]), "chunk %d" % t
+    assert caches[0].state() == caches[1].state()
+    assert torch.equal(caches[0].k, caches[1].k) and torch.equal(caches[0].v, caches[1].v)
+    assert torch.equal(caches[0].k_pool, caches[1].k_pool)
+
+
+def test_host_pipeline_rejects_device_and_pageable_tensors(lc):
+    cache = lc.KVCache(1, 1, 4, 8, 8, 128)
+    step = lc.StreamingStep(cache, 2, lc.SelectParams(top_k=1))
+    pipe = lc.HostPipeline(step)
+    shp = (1, 1, 2, 8, 8, 128)
+    pinned = [torch.zeros(shp, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
+    with pytest.raises(ValueError):
+        pipe.submit(pinned[0].cuda(), *pinned[1:])
+    with pytest.raises(ValueError):
+        pipe.submit(torch.zeros(shp, dtype=torch.bfloat16), *pinned[1:])
+
+
 @pytest.mark.parametrize("first,q_frames", [(1, 1), (3, 3), (5, 2)])
 def test_odd_first_chunk_partial_blocks(lc, first, q_frames):
     """A stream whose first chunk has an odd frame count: the oldest key block
