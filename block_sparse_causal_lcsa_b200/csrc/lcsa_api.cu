@@ -512,21 +512,12 @@ lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames, const lcs
   if (kv->D == 128) score_kernel<128><<<sgrid, SC_THREADS, score_smem_bytes(128), cs>>>(p);
   else score_kernel<64><<<sgrid, SC_THREADS, score_smem_bytes(64), cs>>>(p);
   if ((s = launched()) != LCSA_OK) return s;
-  // one CTA per query block, one key per thread up to 1024 candidates, two beyond
-  const int slots = c_stride <= 1024 ? 1 : 2;
-  const unsigned tthreads = static_cast<unsigned>(((c_stride + slots - 1) / slots + 31) / 32 * 32);
-  if (rows >= 16 * static_cast<int64_t>(g_sm_count[dev])) {
-    // enough rows for four warps per SM sub-partition: a warp per row, no barriers
-    const unsigned wgrid = static_cast<unsigned>((rows + TKW_WARPS - 1) / TKW_WARPS);
-    if (c_stride <= 256) topk_warp_kernel<8><<<wgrid, TKW_WARPS * 32, 0, cs>>>(p);
-    else if (c_stride <= 512) topk_warp_kernel<16><<<wgrid, TKW_WARPS * 32, 0, cs>>>(p);
-    else if (c_stride <= 1024) topk_warp_kernel<32><<<wgrid, TKW_WARPS * 32, 0, cs>>>(p);
-    else topk_warp_kernel<64><<<wgrid, TKW_WARPS * 32, 0, cs>>>(p);
-  } else if (slots == 1) {
-    topk_kernel<1><<<static_cast<unsigned>(rows), tthreads, 0, cs>>>(p);
-  } else {
-    topk_kernel<2><<<static_cast<unsigned>(rows), tthreads, 0, cs>>>(p);
-  }
+  // a warp per query block, the row's keys in its registers
+  const unsigned wgrid = static_cast<unsigned>((rows + TKW_WARPS - 1) / TKW_WARPS);
+  if (c_stride <= 256) topk_warp_kernel<8><<<wgrid, TKW_WARPS * 32, 0, cs>>>(p);
+  else if (c_stride <= 512) topk_warp_kernel<16><<<wgrid, TKW_WARPS * 32, 0, cs>>>(p);
+  else if (c_stride <= 1024) topk_warp_kernel<32><<<wgrid, TKW_WARPS * 32, 0, cs>>>(p);
+  else topk_warp_kernel<64><<<wgrid, TKW_WARPS * 32, 0, cs>>>(p);
   return launched();
 }
 

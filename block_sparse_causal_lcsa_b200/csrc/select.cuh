@@ -15,9 +15,9 @@
 //   float64 value as the definition, bit for bit. Scores are stored as
 //   order-preserving 64-bit keys; candidates outside the row's window get
 //   key 0, below every finite score.
-// topk_kernel   one CTA per query block, one or two keys per thread held in
+// topk_warp_kernel  one warp per query block, the row's keys held in
 //   registers (at most 2048 causal candidates): the exact K-th largest key by
-//   a 1-bit radix select (one CTA-wide count per bit from the top, stopping
+//   a 1-bit radix select (one warp-wide count per bit from the top, stopping
 //   once a single key matches), then one ascending pass keeps every block
 //   above tau+eps and the lowest-index blocks of the band [tau-eps, tau+eps].
 #pragma once
@@ -230,132 +230,12 @@ score_kernel(const __grid_constant__ SelectParams p) {
   }
 }
 
-// Exclusive prefix count of f over the CTA in thread order, and its total.
-__device__ __forceinline__ int cta_excl_count(bool f, int& total, int* wsum) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwarps = blockDim.x >> 5;
-  const uint32_t m = __ballot_sync(0xffffffffu, f);
-  if (lane == 0) wsum[warp] = __popc(m);
-  __syncthreads();
-  int before = 0, tot = 0;
-  for (int w = 0; w < nwarps; ++w) {
-    const int v = wsum[w];
-    before += w < warp ? v : 0;
-    tot += v;
-  }
-  __syncthreads();  // wsum is reused by the next call
-  total = tot;
-  return before + __popc(m & ((1u << lane) - 1u));
-}
-
-// One CTA per query block; candidate j = s*blockDim.x + threadIdx.x sits in
-// slot s of that thread (a row has at most SLOTS*blockDim.x candidates).
-template <int SLOTS>
-__global__ void __launch_bounds__(1024)
-topk_kernel(const __grid_constant__ SelectParams p) {
-  __shared__ int wsum[32];
-  __shared__ uint64_t last_key;
-  const int HbWb = p.Hb * p.Wb;
-  const int nQB = p.nQT * HbWb;
-  const int tid = threadIdx.x, nt = blockDim.x;
-  const int64_t row = blockIdx.x;
-  const int bh = static_cast<int>(row / nQB);
-  const int qi = static_cast<int>(row % nQB);
-  const int tq = qi / HbWb, sp = qi % HbWb;
-  const StreamGeom g = stream_geom(p, bh / p.H, tq);
-  const int ncand = g.ncand;
-  if (ncand > SLOTS * nt) {  // the launch is sized for the longest stream
-    if (tid == 0) atomicOr(p.err, DEVERR_BOUNDS);
-    return;
-  }
-  int y0, y1, x0, x1;
-  window_bounds(sp / p.Wb, p.Hb, p.window, p.window_mode, y0, y1);
-  window_bounds(sp % p.Wb, p.Wb, p.window, p.window_mode, x0, x1);
-  const int C = (g.tq_kv + 1) * (y1 - y0) * (x1 - x0);
-  int K;
-  if (p.top_k > 0) {
-    K = min(C, p.top_k);
-  } else {
-    const double kd = ceil(__dmul_rn(p.density, static_cast<double>(C)));
-    K = min(C, max(1, static_cast<int>(kd)));
-  }
-  const uint64_t* krow = p.keys + row * p.c_stride;
-  if (tid == 0) last_key = 0ull;  // ordered by the counting barriers below
-  uint64_t key[SLOTS];
-  bool act[SLOTS];
-  int nact = 0;
-#pragma unroll
-  for (int s = 0; s < SLOTS; ++s) {
-    const int j = s * nt + tid;
-    key[s] = j < ncand ? krow[j] : 0ull;
-    act[s] = key[s] != 0ull;  // window-masked candidates are not ranked
-    nact += __syncthreads_count(act[s]);
-  }
-
-  // Exact K-th largest key, one bit at a time from the top: the CTA counts
-  // the still-matching keys that have the bit set; the K-th largest has it
-  // iff at least krem of them do. Stops early once one key remains.
-  uint64_t prefix = 0;
-  int krem = K;
-  int bit = 63;
-  for (; bit >= 0 && nact > 1; --bit) {
-    int cnt = 0;
-#pragma unroll
-    for (int s = 0; s < SLOTS; ++s) cnt += __syncthreads_count(act[s] && ((key[s] >> bit) & 1ull));
-    const uint64_t chosen = cnt >= krem ? 1ull : 0ull;
-    if (chosen) {
-      nact = cnt;
-    } else {
-      krem -= cnt;
-      nact -= cnt;
-    }
-    prefix |= chosen << bit;
-#pragma unroll
-    for (int s = 0; s < SLOTS; ++s) act[s] = act[s] && ((key[s] >> bit) & 1ull) == chosen;
-  }
-  if (bit >= 0) {  // a single key matches the prefix: it is the K-th largest
-#pragma unroll
-    for (int s = 0; s < SLOTS; ++s)
-      if (act[s]) last_key = key[s];
-    __syncthreads();
-    prefix = last_key;
-  }
-  const double tau = key_value(prefix);
-  const uint64_t k_hi = order_key(__dadd_rn(tau, p.tie_eps));
-  const uint64_t k_lo = order_key(__dsub_rn(tau, p.tie_eps));
-  int above = 0;
-#pragma unroll
-  for (int s = 0; s < SLOTS; ++s) above += __syncthreads_count(key[s] > k_hi);
-  const int need = K - above;
-
-  // Keep everything above the band and the lowest-index band members; write
-  // the kept ids in ascending order.
-  int32_t* out = p.blk_idx + row * p.kmax;
-  int n_band = 0, n_sel = 0;
-#pragma unroll
-  for (int s = 0; s < SLOTS; ++s) {
-    const int j = s * nt + tid;
-    const bool in_above = key[s] > k_hi;
-    const bool in_band = key[s] >= k_lo && key[s] <= k_hi;
-    int band_tot, sel_tot;
-    const int band_before = cta_excl_count(in_band, band_tot, wsum);
-    const bool take = in_above || (in_band && n_band + band_before < need);
-    const int pos = n_sel + cta_excl_count(take, sel_tot, wsum);
-    if (take) {
-      if (pos < p.kmax) out[pos] = j;
-      else atomicOr(p.err, DEVERR_BOUNDS);
-    }
-    n_band += band_tot;
-    n_sel += sel_tot;
-  }
-  for (int pos = K + tid; pos < p.kmax; pos += nt) out[pos] = -1;
-  if (tid == 0) p.blk_cnt[row] = K;
-}
-
-// One warp per query block (4 per CTA), for launches with many rows: the
-// row's keys sit in registers (candidate j = 32*i + lane in slot i, at most
-// 32*KPL candidates) and each radix pass is one ballot per slot, with no
-// CTA-wide barrier; the same selection as topk_kernel.
+// One warp per query block (4 per CTA): the row's keys sit in registers as
+// 32-bit halves (candidate j = 32*i + lane in slot i, at most 32*KPL
+// candidates). The K-th largest key is found one bit at a time, first over
+// the high halves, then - only if several keys share the K-th largest high
+// half - over the low halves of those keys; a bit's count is one compare per
+// slot and lane and one warp-wide add, with no barrier.
 constexpr int TKW_WARPS = 4;
 template <int KPL>
 __global__ void __launch_bounds__(TKW_WARPS * 32)
@@ -387,62 +267,95 @@ topk_warp_kernel(const __grid_constant__ SelectParams p) {
   }
   const uint64_t* krow = p.keys + row * p.c_stride;
   const int nslots = (ncand + 31) / 32;
-  uint64_t key[KPL];
-  bool act[KPL];
-  int nact = 0;
+  uint32_t hi[KPL], lo[KPL];
+  int lc = 0;
 #pragma unroll
   for (int i = 0; i < KPL; ++i) {
     const int j = 32 * i + lane;
-    key[i] = (i < nslots && j < ncand) ? krow[j] : 0ull;
-    act[i] = key[i] != 0ull;                   // window-masked candidates are not ranked
-    if (i < nslots) nact += __popc(__ballot_sync(0xffffffffu, act[i]));
+    const uint64_t k = (i < nslots && j < ncand) ? krow[j] : 0ull;
+    hi[i] = static_cast<uint32_t>(k >> 32);
+    lo[i] = static_cast<uint32_t>(k);
+    lc += k != 0ull;                           // window-masked candidates (key 0) are not ranked
   }
-  // exact K-th largest key, one bit at a time from the top (as topk_kernel)
-  uint64_t prefix = 0;
+  // nact: unmasked keys that match the prefix found so far. A masked key has
+  // no bit set, so it never matches a prefix extended by a set bit and is
+  // never counted.
+  int nact = __reduce_add_sync(0xffffffffu, lc);
   int krem = K;
-  int bit = 63;
+  uint32_t phi = 0, plo = 0;
+  int bit = 31;
   for (; bit >= 0 && nact > 1; --bit) {
-    int cnt = 0;
+    const uint32_t t = (phi >> bit) | 1u;
+    lc = 0;
 #pragma unroll
-    for (int i = 0; i < KPL; ++i) {
-      if (i >= nslots) break;
-      cnt += __popc(__ballot_sync(0xffffffffu, act[i] && ((key[i] >> bit) & 1ull)));
-    }
-    const uint64_t chosen = cnt >= krem ? 1ull : 0ull;
-    if (chosen) {
+    for (int i = 0; i < KPL; ++i)
+      if (i < nslots) lc += (hi[i] >> bit) == t;
+    const int cnt = __reduce_add_sync(0xffffffffu, lc);
+    if (cnt >= krem) {
       nact = cnt;
+      phi |= 1u << bit;
     } else {
       krem -= cnt;
       nact -= cnt;
     }
-    prefix |= chosen << bit;
-#pragma unroll
-    for (int i = 0; i < KPL; ++i) act[i] = act[i] && ((key[i] >> bit) & 1ull) == chosen;
   }
-  if (bit >= 0) {  // a single key matches the prefix: it is the K-th largest
-    uint64_t found = 0ull;
+  // bits of the high half above hbit are decided (all of them when hbit = -1)
+  const int hbit = bit;
+  int lbit = 32;
+  if (nact > 1) {
+    // several keys share the K-th largest high half: rank their low halves
+    for (bit = 31; bit >= 0 && nact > 1; --bit) {
+      const uint32_t t = (plo >> bit) | 1u;
+      lc = 0;
+#pragma unroll
+      for (int i = 0; i < KPL; ++i)
+        if (i < nslots) lc += hi[i] == phi && (lo[i] >> bit) == t;
+      const int cnt = __reduce_add_sync(0xffffffffu, lc);
+      if (cnt >= krem) {
+        nact = cnt;
+        plo |= 1u << bit;
+      } else {
+        krem -= cnt;
+        nact -= cnt;
+      }
+    }
+    lbit = bit;
+  }
+  uint64_t kth = (static_cast<uint64_t>(phi) << 32) | plo;
+  if (lbit >= 0) {
+    // a single unmasked key matches the decided bits: it is the K-th largest
+    uint32_t fh = 0, fl = 0;
+    bool have = false;
 #pragma unroll
     for (int i = 0; i < KPL; ++i) {
       if (i >= nslots) break;
-      const uint32_t m = __ballot_sync(0xffffffffu, act[i]);
+      const bool nz = (hi[i] | lo[i]) != 0u;
+      bool m;
+      if (lbit == 32) {
+        m = nz && (hbit + 1 >= 32 || (hi[i] >> (hbit + 1)) == (phi >> (hbit + 1)));
+      } else {
+        m = hi[i] == phi && (lbit + 1 >= 32 || (lo[i] >> (lbit + 1)) == (plo >> (lbit + 1)));
+      }
       if (m) {
-        const int src = __ffs(m) - 1;
-        found = (static_cast<uint64_t>(__shfl_sync(0xffffffffu, static_cast<uint32_t>(key[i] >> 32), src)) << 32) |
-                __shfl_sync(0xffffffffu, static_cast<uint32_t>(key[i]), src);
+        fh = hi[i];
+        fl = lo[i];
+        have = true;
       }
     }
-    prefix = found;
+    const uint32_t who = __ballot_sync(0xffffffffu, have);
+    if (who != 0u) {
+      const int src = __ffs(who) - 1;
+      kth = (static_cast<uint64_t>(__shfl_sync(0xffffffffu, fh, src)) << 32) | __shfl_sync(0xffffffffu, fl, src);
+    }
   }
-  const double tau = key_value(prefix);
+  const double tau = key_value(kth);
   const uint64_t k_hi = order_key(__dadd_rn(tau, p.tie_eps));
   const uint64_t k_lo = order_key(__dsub_rn(tau, p.tie_eps));
-  int above = 0;
+  lc = 0;
 #pragma unroll
-  for (int i = 0; i < KPL; ++i) {
-    if (i >= nslots) break;
-    above += __popc(__ballot_sync(0xffffffffu, key[i] > k_hi));
-  }
-  const int need = K - above;
+  for (int i = 0; i < KPL; ++i)
+    if (i < nslots) lc += ((static_cast<uint64_t>(hi[i]) << 32) | lo[i]) > k_hi;
+  const int need = K - __reduce_add_sync(0xffffffffu, lc);
   int32_t* out = p.blk_idx + row * p.kmax;
   const uint32_t lt_mask = (1u << lane) - 1u;
   int n_band = 0, n_sel = 0;
@@ -450,8 +363,9 @@ topk_warp_kernel(const __grid_constant__ SelectParams p) {
   for (int i = 0; i < KPL; ++i) {
     if (i >= nslots) break;
     const int j = 32 * i + lane;
-    const bool in_above = key[i] > k_hi;
-    const bool in_band = key[i] >= k_lo && key[i] <= k_hi;
+    const uint64_t k = (static_cast<uint64_t>(hi[i]) << 32) | lo[i];
+    const bool in_above = k > k_hi;
+    const bool in_band = k >= k_lo && k <= k_hi;
     const uint32_t band_mask = __ballot_sync(0xffffffffu, in_band);
     const bool take = in_above || (in_band && (n_band + __popc(band_mask & lt_mask)) < need);
     const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
