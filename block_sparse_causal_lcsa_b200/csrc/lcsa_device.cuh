@@ -59,6 +59,23 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
+// The same test, but a thread whose phase is not complete is suspended by the
+// hardware until it completes or `hint_ns` pass, instead of returning at once:
+// a waiting warp then takes no issue slots from the warps it shares a
+// sub-partition with (the softmax warps share theirs with the TMA producers
+// and the MMA issuer).
+__device__ __forceinline__ bool mbar_test_suspend(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return done != 0;
+}
+
 // Context of the bounded waits of one CTA.
 struct WaitCtx {
   uint64_t limit_ns;       // give up after this long without progress
@@ -68,19 +85,19 @@ struct WaitCtx {
 
 // Wait for the phase of `bar` with parity `parity` to complete. Returns false
 // (and raises the CTA's abort flag) if the limit ran out or another role of
-// the CTA already aborted.
+// the CTA already aborted. Each unsuccessful test suspends the thread for at
+// most WAIT_SUSPEND_NS, so the limit is checked at least that often.
+constexpr uint32_t WAIT_SUSPEND_NS = 100000;
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const WaitCtx& w) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_test(bar, parity)) return true;
-    if ((it & 31u) == 0u) {
-      if (*w.abort) return false;
-      if (global_ns() - t0 > w.limit_ns) {
-        atomicOr(w.err, DEVERR_TIMEOUT);
-        *w.abort = 1;
-        return false;
-      }
+  for (;;) {
+    if (mbar_test_suspend(bar, parity, WAIT_SUSPEND_NS)) return true;
+    if (*w.abort) return false;
+    if (global_ns() - t0 > w.limit_ns) {
+      atomicOr(w.err, DEVERR_TIMEOUT);
+      *w.abort = 1;
+      return false;
     }
   }
 }
