@@ -1,0 +1,55 @@
+"""Host-side arithmetic behind bench.py's JSON line (no GPU): the FLOP count
+that the roofline divides by, and the whole-job throughput across ranks."""
+import importlib.util
+import os
+
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+class _Cache:
+    """Just the cache state attn_flops reads: the first cached frame of each stream."""
+
+    def __init__(self, begins):
+        self._begins = begins
+
+    def begin(self, b):
+        return self._begins[b]
+
+
+def test_attn_flops_counts_kept_key_tokens():
+    bench = _bench()
+    Hb, Wb, D = 2, 3, 128
+    # one stream, one head, two query blocks keeping 3 and 2 blocks (-1 = unused slot)
+    cnt = torch.tensor([[[3, 2]]], dtype=torch.int32)
+    idx = torch.tensor([[[[0, 4, 7], [2, 9, -1]]]], dtype=torch.int32)
+    full = bench.attn_flops(cnt, idx, _Cache([4]), Hb, Wb, D)
+    assert full == 4.0 * D * 128 * (5 * 128)
+    # an odd first cached frame leaves the oldest key block (ids < Hb*Wb) with one
+    # frame: kept blocks 0, 4 and 2 then hold 64 keys each; the -1 slot is not counted
+    partial = bench.attn_flops(cnt, idx, _Cache([3]), Hb, Wb, D)
+    assert partial == 4.0 * D * 128 * (5 * 128 - 3 * 64)
+
+
+def test_attn_flops_sums_streams_separately():
+    bench = _bench()
+    cnt = torch.tensor([[[1]], [[1]]], dtype=torch.int32)
+    idx = torch.tensor([[[[0]]], [[[0]]]], dtype=torch.int32)
+    # stream 0 starts on an even frame (full block), stream 1 on an odd one (one frame)
+    f = bench.attn_flops(cnt, idx, _Cache([2, 1]), 1, 1, 64)
+    assert f == 4.0 * 64 * 128 * (128 + 64)
+
+
+def test_whole_job_throughput_divides_by_every_rank_chunk():
+    bench = _bench()
+    # 4 ranks, 13 chunks each, slowest rank 26 ms: 0.5 ms per chunk of the whole job
+    assert bench.whole_job_ms_per_chunk(26.0, 13, 4) == 0.5
+    assert bench.whole_job_ms_per_chunk(0.25, 1, 1) == 0.25
