@@ -34,3 +34,4 @@ from .api import (  # noqa: F401
     tensor_desc,
 )
 from .build import LIB_PATH  # noqa: F401
+from .partition import rank_slices, rank_units  # noqa: F401

@@ -182,24 +182,51 @@ def select_workspace_bytes(cache: KVCache, q_frames: int) -> int:
     return int(_lib.lcsa_select_workspace_bytes(C.byref(cache.struct), q_frames))
 
 
+def _check_select_io(q_pool: torch.Tensor, q_frames: int, cache: KVCache, kmax: int,
+                     blk_idx: torch.Tensor, blk_cnt: torch.Tensor) -> None:
+    """The C call writes blk_idx / blk_cnt and reads q_pool by the cache's
+    extents: reject anything whose dtype, shape, layout or device would let
+    the kernels read or write past a tensor (ValueError, nothing launched)."""
+    nQT = (q_frames + 1) // 2
+    Hb, Wb = cache.Y // 8, cache.X // 8
+    nQB = nQT * Hb * Wb
+    want = {"q_pool": (q_pool, torch.float64, (cache.B, cache.H, nQT, Hb, Wb, cache.D)),
+            "blk_idx": (blk_idx, torch.int32, (cache.B, cache.H, nQB, kmax)),
+            "blk_cnt": (blk_cnt, torch.int32, (cache.B, cache.H, nQB))}
+    for name, (t, dtype, shape) in want.items():
+        if not isinstance(t, torch.Tensor):
+            raise ValueError("%s must be a tensor" % name)
+        if t.dtype != dtype:
+            raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+        if tuple(t.shape) != shape:
+            raise ValueError("%s must have shape %s for this cache, got %s" % (name, shape, tuple(t.shape)))
+        if not t.is_contiguous():
+            raise ValueError("%s must be contiguous" % name)
+    dev = cache.k.device
+    for name, (t, _, _) in want.items():
+        if not t.is_cuda or t.device != dev:
+            raise ValueError("%s must be a CUDA tensor on the cache's device %s, got %s" % (name, dev, t.device))
+
+
 def select_blocks(q_pool: torch.Tensor, q_frames: int, cache: KVCache, params: SelectParams,
                   kmax: Optional[int] = None, blk_idx: Optional[torch.Tensor] = None,
                   blk_cnt: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                   stream: Optional[torch.cuda.Stream] = None):
     """Top-K key blocks of every query block: (blk_idx [B,H,nQB,kmax], blk_cnt [B,H,nQB])."""
     if kmax is None:
-        kmax = select_kmax(cache, q_frames, params)
+        kmax = blk_idx.shape[-1] if blk_idx is not None else select_kmax(cache, q_frames, params)
+    nQB = ((q_frames + 1) // 2) * (cache.Y // 8) * (cache.X // 8)
+    dev = q_pool.device
+    if blk_idx is None:
+        blk_idx = torch.empty((cache.B, cache.H, nQB, kmax), dtype=torch.int32, device=dev)
+    if blk_cnt is None:
+        blk_cnt = torch.empty((cache.B, cache.H, nQB), dtype=torch.int32, device=dev)
+    _check_select_io(q_pool, q_frames, cache, kmax, blk_idx, blk_cnt)
     need = select_workspace_bytes(cache, q_frames)
     if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_pool.device)
-    B, H, nQT, Hb, Wb, D = q_pool.shape
-    if not q_pool.is_contiguous() or q_pool.dtype != torch.float64:
-        raise ValueError("q_pool must be contiguous float64")
-    nQB = nQT * Hb * Wb
-    if blk_idx is None:
-        blk_idx = torch.empty((B, H, nQB, kmax), dtype=torch.int32, device=q_pool.device)
-    if blk_cnt is None:
-        blk_cnt = torch.empty((B, H, nQB), dtype=torch.int32, device=q_pool.device)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    elif not workspace.is_cuda or workspace.device != cache.k.device or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor on the cache's device")
     sp = params.struct(kmax)
     _check(_lib.lcsa_select_blocks(q_pool.data_ptr(), q_frames, C.byref(cache.struct), C.byref(sp),
                                    blk_idx.data_ptr(), blk_cnt.data_ptr(), workspace.data_ptr(),
@@ -214,13 +241,14 @@ def select_blocks_noalloc(q_pool: torch.Tensor, q_frames: int, cache: KVCache, p
     """select_blocks into caller-given outputs, with the library's fixed
     scratch array in place of a workspace: nothing is allocated, so it suits
     callers that may not allocate device memory while they run. kmax is
-    blk_idx.shape[-1]. Raises LcsaError(ERR_SCRATCH_LIMIT) when the selection
-    needs more than SELECT_STATIC_SCRATCH_BYTES of scratch; calls that overlap
-    on the GPU share that scratch and must be serialised."""
-    if q_pool.dtype != torch.float64 or not q_pool.is_contiguous():
-        raise ValueError("q_pool must be contiguous float64")
-    if not blk_idx.is_contiguous() or not blk_cnt.is_contiguous():
-        raise ValueError("blk_idx and blk_cnt must be contiguous")
+    blk_idx.shape[-1]; q_pool must be float64 [B,H,nQT,Y/8,X/8,D] and the
+    outputs int32 [B,H,nQB,kmax] / [B,H,nQB] on the cache's device (else
+    ValueError). Raises LcsaError(ERR_SCRATCH_LIMIT) when the selection needs
+    more than SELECT_STATIC_SCRATCH_BYTES of scratch; calls that overlap on
+    the GPU share that scratch and must be serialised."""
+    if not isinstance(blk_idx, torch.Tensor) or blk_idx.dim() != 4:
+        raise ValueError("blk_idx must be an int32 tensor [B,H,nQB,kmax]")
+    _check_select_io(q_pool, q_frames, cache, blk_idx.shape[-1], blk_idx, blk_cnt)
     sp = params.struct(blk_idx.shape[-1])
     _check(_lib.lcsa_select_blocks_noalloc(q_pool.data_ptr(), q_frames, C.byref(cache.struct),
                                            C.byref(sp), blk_idx.data_ptr(), blk_cnt.data_ptr(),

@@ -290,8 +290,9 @@ LCSA_API lcsa_status lcsa_select_blocks(const double* q_pool, int32_t q_frames,
  * Limit: lcsa_select_workspace_bytes(kv, q_frames) must not exceed
  * LCSA_SELECT_STATIC_SCRATCH_BYTES, else LCSA_ERR_SCRATCH_LIMIT, returned
  * before any device work. Four streams of 768x1408 frames (12 heads, an
- * 8-frame cache) need 6.7 MB and fit; one 1536x2816 stream with a 6-frame
- * cache needs 18.3 MB and does not.
+ * 8-frame cache) need 6.7 MB and fit; one 1536x2688 stream with a 6-frame
+ * cache (12 heads x 252 query blocks x 756 candidates) needs 18.3 MB and
+ * does not.
  * Other errors are those of lcsa_select_blocks (LCSA_ERR_CUDA also if the
  * address look-up fails).
  */
@@ -423,9 +424,11 @@ LCSA_API lcsa_status lcsa_sparse_attn_bwd(const lcsa_tensor* q, const lcsa_kv_ca
 LCSA_API lcsa_status lcsa_last_device_error(lcsa_stream_t stream);
 
 /*
- * Test hook: make the next kernel launches of the library on the current
- * device see a wait limit of `ns` nanoseconds (0 restores the default of
- * about one second). Used to exercise the timeout path without any fault.
+ * Test hook: make the library's next kernel launches, on every device and
+ * from every host thread of the process (the limit is one process-wide
+ * setting, not a per-device one), see a wait limit of `ns` nanoseconds (0
+ * restores the default of about one second). Used to exercise the timeout
+ * path without any fault.
  */
 LCSA_API lcsa_status lcsa_debug_set_wait_limit_ns(uint64_t ns);
 
@@ -438,10 +441,11 @@ LCSA_API lcsa_status lcsa_debug_set_wait_limit_ns(uint64_t ns);
 LCSA_API lcsa_status lcsa_debug_stalled_wait(uint64_t limit_ns, lcsa_stream_t stream);
 
 /*
- * Test hook: y[i] = 2^x[i] (x[i] <= 8) evaluated with the polynomial the
- * attention kernel uses on the FMA pipe for a quarter of its exponentials
- * (range reduction x = n + f, |f| <= 1/2, degree-3 minimax polynomial for
- * 2^f, exponent add for 2^n). x, y: device float32 arrays of n elements.
+ * Test hook: y[i] = 2^x[i] (x[i] <= 8) evaluated with the FMA-pipe
+ * polynomial that the attention softmax can use in place of the
+ * special-function unit for part of its exponentials (range reduction
+ * x = n + f, |f| <= 1/2, degree-3 minimax polynomial for 2^f, exponent add
+ * for 2^n). x, y: device float32 arrays of n elements.
  */
 LCSA_API lcsa_status lcsa_debug_exp2_poly(const float* x, float* y, int64_t n,
                                           lcsa_stream_t stream);

@@ -8,13 +8,14 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
-    # The built library is not committed: a fresh checkout compiles it once
-    # (loaded by path, since importing the package needs the library).
+    # The built library is not committed, and one carried over from another
+    # checkout may predate its sources: rebuild whenever any source is newer
+    # than liblcsa.so (loaded by path, since importing the package needs the
+    # library).
     import importlib.util
 
     spec = importlib.util.spec_from_file_location(
         "lcsa_build", os.path.join(ROOT, "block_sparse_causal_lcsa_b200", "build.py"))
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
-    if not os.path.exists(mod.LIB_PATH):
-        mod.build()
+    mod.build()

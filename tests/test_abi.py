@@ -183,3 +183,38 @@ def test_select_kmax_covers_every_row(lib, mode, window):
         Ks.append(orc.top_k_count(C_i, 0, 0.136))
     assert kmax >= max(Ks)
     assert kmax <= max(Ks) + 1 or mode >= 2
+
+
+def test_binding_rejects_bad_selection_outputs(lib):
+    """The Python binding checks dtype, shape, layout and device of q_pool and
+    of caller-given blk_idx / blk_cnt before calling the library, so a wrong
+    output can never be written past its end (ValueError, nothing launched)."""
+    import torch
+    import block_sparse_causal_lcsa_b200 as lc
+
+    cache = lc.KVCache(1, 2, 6, 16, 24, 128, device="cpu")
+    cache.struct.begin[0], cache.struct.end[0] = 0, 6
+    params = lc.SelectParams(density=0.5)
+    nQB, kmax = 1 * 2 * 3, 40
+    good = dict(q_pool=torch.zeros((1, 2, 1, 2, 3, 128), dtype=torch.float64),
+                blk_idx=torch.zeros((1, 2, nQB, kmax), dtype=torch.int32),
+                blk_cnt=torch.zeros((1, 2, nQB), dtype=torch.int32))
+    bad = [
+        dict(blk_idx=good["blk_idx"].long()),                                    # int64 outputs
+        dict(blk_cnt=good["blk_cnt"].long()),
+        dict(blk_idx=torch.zeros((1, 2, nQB - 1, kmax), dtype=torch.int32)),     # too few rows
+        dict(blk_cnt=torch.zeros((1, 2, nQB - 1), dtype=torch.int32)),
+        dict(blk_idx=torch.zeros((1, 2, kmax, nQB), dtype=torch.int32).transpose(2, 3)),  # not contiguous
+        dict(q_pool=good["q_pool"].float()),                                     # float32 pooled Q
+        dict(q_pool=torch.zeros((1, 2, 2, 2, 3, 128), dtype=torch.float64)),     # q_pool of 2 time blocks
+        dict(blk_idx=[0] * 10),                                                  # not a tensor
+        {},                                                                      # right shapes, host memory
+    ]
+    for b in bad:
+        a = {**good, **b}
+        with pytest.raises(ValueError):
+            lc.select_blocks_noalloc(a["q_pool"], 2, cache, params, a["blk_idx"], a["blk_cnt"])
+        if isinstance(a["blk_idx"], torch.Tensor) and a["blk_idx"].dim() == 4:
+            with pytest.raises(ValueError):
+                lc.select_blocks(a["q_pool"], 2, cache, params, a["blk_idx"].shape[-1], a["blk_idx"],
+                                 a["blk_cnt"], workspace=torch.zeros(16, dtype=torch.uint8))

@@ -53,3 +53,44 @@ def test_whole_job_throughput_divides_by_every_rank_chunk():
     # 4 ranks, 13 chunks each, slowest rank 26 ms: 0.5 ms per chunk of the whole job
     assert bench.whole_job_ms_per_chunk(26.0, 13, 4) == 0.5
     assert bench.whole_job_ms_per_chunk(0.25, 1, 1) == 0.25
+
+
+class _CacheSpan:
+    """begin / end frames per stream, as bench.allowed_pairs reads them."""
+
+    def __init__(self, spans):
+        self._s = spans
+
+    def begin(self, b):
+        return self._s[b][0]
+
+    def end(self, b):
+        return self._s[b][1]
+
+
+def test_allowed_pairs_equals_the_oracles_candidate_counts():
+    """The selection's float64 work is counted from the pairs the coarse map
+    scores; for every window mode that count equals the sum of the oracle's
+    per-row candidate counts C_i."""
+    import numpy as np
+    import lcsa_inputs as li
+    from oracle import lcsa_oracle as orc
+
+    bench = _bench()
+    w = li.workload("chunk")
+    assert bench.allowed_pairs(w, _CacheSpan([(0, 6)])) == 12 * 66 * 198
+    for window, mode in [(0, 0), (3, 0), (3, 1), (5, 0), (20, 2), (20, 3), (35, 2)]:
+        w = li.Workload("pairs", B=2, H=1, D=64, Y=40, X=56, q_frames=2, kv_past=(4, 3), cap_frames=6,
+                        density=0.2, window=window, window_mode=mode, seed=3)
+        spans = [(0, 6), (1, 6)]
+        got = bench.allowed_pairs(w, _CacheSpan(spans))
+        want = 0
+        for lo, hi in spans:
+            F = hi - lo
+            nKT = (F + 1) // 2
+            qp = np.zeros((w.Hb * w.Wb, w.D))
+            kp = np.zeros((nKT * w.Hb * w.Wb, w.D))
+            _, _, Cs = orc.select_head(qp, kp, w.q_frames, F, w.Y, w.X, density=w.density,
+                                       window=window, mode=mode)
+            want += int(Cs.sum())
+        assert got == want, (window, mode, got, want)

@@ -5,8 +5,10 @@ Tolerance (derived from the arithmetic): Q, K, V, dO are bf16 and exact in
 both paths; the GPU rounds P and dS to bf16 (relative error 2^-9) before their
 tensor-core products, accumulates in fp32 and rounds dQ, dK, dV to bf16
 (2^-9). Summed over hundreds to thousands of keys these independent rounding
-errors give a relative L2 error of a few 1e-3; the bar is rel-L2 <= 2e-2 per
-tensor, with max-abs <= 5e-2 of the tensor's largest magnitude."""
+errors give a relative L2 error of a few 1e-3 (measured on these cases: at
+most 3.3e-3 rel-L2 and 5.5e-3 max-abs over the tensor's largest magnitude);
+the bar is rel-L2 <= 5e-3 per tensor, with max-abs <= 1e-2 of the tensor's
+largest magnitude, so a change that doubled the gradient error fails."""
 import numpy as np
 import pytest
 import torch
@@ -16,8 +18,8 @@ from oracle import lcsa_oracle as orc
 
 pytestmark = pytest.mark.gpu
 
-REL_L2 = 2e-2
-MAX_REL = 5e-2
+REL_L2 = 5e-3
+MAX_REL = 1e-2
 
 
 @pytest.fixture(scope="module")
@@ -36,6 +38,7 @@ def _errs(got, ref):
 
 def _check(got, ref, where):
     rel, mx = _errs(got, ref)
+    print("%s rel-L2 %.3g max-abs/max %.3g" % (where, rel, mx))
     assert rel <= REL_L2 and mx <= MAX_REL, "%s rel-L2 %.3g max-abs/max %.3g" % (where, rel, mx)
     return rel, mx
 

@@ -49,21 +49,27 @@ def test_small_workloads_every_row(lc, w):
 
 
 FULL = ["chunk", "multistream", "uhr_truncate", "uhr_preserve"]
+# workloads whose O is compared on every query block of the checked heads (the
+# oracle does 66 query blocks of a 768x1408 head in seconds); the 1536x2688
+# ones on 8 sampled query blocks
+FULL_O_ALL_ROWS = {"chunk", "multistream"}
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_selection_all_rows_output_sampled(lc, name):
+def test_full_size_selection_all_rows_output_checked(lc, name):
     w = li.workload(name)
     x = li.make_inputs(w)
     g = run_gpu(lc, w, x)
     assert g["err"] == 0
     rng = np.random.default_rng(11)
     nQB = g["blk_cnt"].shape[2]
-    rows = sorted(rng.choice(nQB, size=6, replace=False).tolist() + [0, nQB - 1])
+    if name in FULL_O_ALL_ROWS:
+        rows = list(range(nQB))
+    else:
+        rows = sorted(rng.choice(nQB, size=6, replace=False).tolist() + [0, nQB - 1])
     heads = [0, w.H - 1]
     for b in range(w.B):
         for h in range(w.H):
-            sel_rows = None if h in heads else rows
             ref = oracle_head(w, x, b, h, rows=rows if h in heads else [])
             where = "%s b%d h%d" % (name, b, h)
             assert np.array_equal(g["q_pool"][b, h].reshape(-1, w.D), ref["q_pool"]), where
@@ -71,11 +77,15 @@ def test_full_size_selection_all_rows_output_sampled(lc, name):
             check_selection(g["blk_idx"][b, h], g["blk_cnt"][b, h], ref["sel"], where)
             if h in heads:
                 check_output(g["O"][b, h], ref["O"], g["LSE"][b, h], ref["LSE"], where)
-            del sel_rows
 
 
-def test_full_clip_selection_and_sampled_output(lc):
-    w = li.workload("clip")
+@pytest.mark.parametrize("name", ["clip_5", "clip", "clip_30"])
+def test_full_clip_selection_and_sampled_output(lc, name):
+    """The whole 101-frame clip at each density of the sweep (5%, 13.6%, 30%):
+    pooled features and every selection row of every head bit for bit; O and
+    LSE of two heads on sampled query blocks, the newest frame pair's (the
+    longest rows: 43, 117 and 258 kept blocks) among them."""
+    w = li.workload(name)
     x = li.make_inputs(w)
     dev = "cuda"
     k = x["k"][0].unsqueeze(0).to(dev)
@@ -85,23 +95,26 @@ def test_full_clip_selection_and_sampled_output(lc):
     cache = lc.KVCache.wrap(k, v, k_pool)
     params = params_of(lc, w)
     idx, cnt = lc.select_blocks(q_pool, w.q_frames, cache, params)
-    o, lse = lc.sparse_attn_fwd(q, cache, idx, cnt)
+    o, lse = lc.sparse_attn_fwd(q, cache, idx, cnt, workspace=lc.attn_workspace(w.D))
     torch.cuda.synchronize()
     assert lc.last_device_error() == 0
     idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
     O, L = o.double().cpu().numpy(), lse.double().cpu().numpy()
     qp, kp = q_pool.cpu().numpy(), k_pool.cpu().numpy()
     nQB = cnt.shape[2]
-    rows = [0, 65, 400, nQB - 66, nQB - 1]
+    HbWb = w.Hb * w.Wb
+    rows = [0, 65, 400, nQB - HbWb, nQB - HbWb // 2, nQB - 1]
+    longest = int(np.ceil(w.density * nQB))
     for h in range(w.H):
         qh, kh = orc.widen(x["q"][0, h]), orc.widen(x["k"][0][h])
         rq, rk = orc.pool_blocks(qh), orc.pool_blocks(kh)
         assert np.array_equal(qp[0, h].reshape(-1, w.D), rq) and np.array_equal(kp[0, h].reshape(-1, w.D), rk)
         sel, Ks, Cs = orc.select_head(rq, rk, w.q_frames, w.q_frames, w.Y, w.X, density=w.density)
-        check_selection(idx[0, h], cnt[0, h], sel, "clip h%d" % h)
+        check_selection(idx[0, h], cnt[0, h], sel, "%s h%d" % (name, h))
+        assert int(cnt[0, h, nQB - 1]) == longest
         if h in (0, 7):
             ro, rl = orc.attend_head(qh, kh, orc.widen(x["v"][0][h]), sel, rows)
-            check_output(O[0, h], ro, L[0, h], rl, "clip h%d" % h)
+            check_output(O[0, h], ro, L[0, h], rl, "%s h%d" % (name, h))
 
 
 @pytest.mark.parametrize("past", [250, 372])
@@ -371,11 +384,23 @@ def test_argument_errors_leave_outputs_untouched(lc):
         lc.select_blocks(step.q_pool, 2, g["cache"], lc.SelectParams(density=0.5, window=4),
                          step.kmax, step.blk_idx, step.blk_cnt)
     assert e.value.status == -1
-    with pytest.raises(lc.LcsaError):
+    # kmax = 1 cannot hold a full-density row: refused by the library
+    idx1 = torch.full(step.blk_idx.shape[:3] + (1,), 5, dtype=torch.int32, device="cuda")
+    cnt1 = torch.full(step.blk_cnt.shape, 5, dtype=torch.int32, device="cuda")
+    with pytest.raises(lc.LcsaError) as e:
+        lc.select_blocks(step.q_pool, 2, g["cache"], lc.SelectParams(density=1.0), 1, idx1, cnt1)
+    assert e.value.status == -4
+    # outputs whose row stride disagrees with kmax, or of the wrong type, are
+    # refused by the binding before any launch
+    with pytest.raises(ValueError):
         lc.select_blocks(step.q_pool, 2, g["cache"], lc.SelectParams(density=1.0), 1,
                          step.blk_idx, step.blk_cnt)
+    with pytest.raises(ValueError):
+        lc.select_blocks_noalloc(step.q_pool, 2, g["cache"], lc.SelectParams(density=0.5),
+                                 step.blk_idx.long(), step.blk_cnt)
     torch.cuda.synchronize()
     assert torch.equal(before, step.blk_idx)
+    assert (idx1 == 5).all() and (cnt1 == 5).all()
 
 
 def test_wait_timeout_reports_and_context_survives(lc):
@@ -404,8 +429,8 @@ def test_out_of_range_block_id_is_reported(lc):
 
 
 def test_exp2_polynomial_error_bound(lc):
-    """The FMA-pipe 2^x used for a quarter of the softmax exponentials stays
-    within its fitted relative error bound (7.5e-5, plus float32 rounding)
+    """The FMA-pipe 2^x that the softmax can use in place of the
+    special-function unit stays within its fitted relative error bound (7.5e-5, plus float32 rounding)
     against torch's float32 exp2, over the softmax's argument range."""
     x = torch.linspace(-100.0, 8.0, 1_000_001, device="cuda", dtype=torch.float32)
     y = lc.debug_exp2_poly(x)

@@ -37,7 +37,7 @@ def _lib():
 
 def test_oversized_request_rejected_before_device_work():
     """A selection that needs more scratch than the fixed array holds (one
-    1536x2816 stream: 12 heads x 252 query blocks x 756 candidates x 8 bytes)
+    1536x2688 stream: 12 heads x 252 query blocks x 756 candidates x 8 bytes)
     is refused with its own status, before any CUDA call (no GPU here)."""
     _abi, lib = _lib()
     kv = _abi.KVCacheStruct()
@@ -89,3 +89,13 @@ def test_noalloc_matches_workspace_select_on_consecutive_calls():
     for (w, _, _, _, ref_idx, ref_cnt), (idx, cnt) in zip(cases, outs):
         assert torch.equal(cnt, ref_cnt), w.name
         assert torch.equal(idx, ref_idx), w.name
+
+    # and once more through the Python binding, which checks the outputs'
+    # dtype, shape and device before the same C call
+    w, cache, q_pool, params, ref_idx, ref_cnt = cases[0]
+    idx = torch.full_like(ref_idx, 7777)
+    cnt = torch.full_like(ref_cnt, 7777)
+    lc.select_blocks_noalloc(q_pool, w.q_frames, cache, params, idx, cnt)
+    torch.cuda.synchronize()
+    assert lc.last_device_error() == 0
+    assert torch.equal(cnt, ref_cnt) and torch.equal(idx, ref_idx)
