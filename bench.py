@@ -77,7 +77,8 @@ def load_peaks():
     if os.path.exists(p):
         d = json.load(open(p))
         return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "sm_max_mhz": d.get("sm_max_mhz"),
+                "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
             "source": "fallback"}
 
@@ -190,67 +191,128 @@ def attn_flops(blk_cnt: torch.Tensor, blk_idx: torch.Tensor, cache, Hb: int, Wb:
 
 
 # ----------------------------------------------------------------------------- our arm
-def run_ours(args, world, rank, local):
-    import block_sparse_causal_lcsa_b200 as lc
+def make_flusher(dev):
+    """L2 flush: write 512 MB, then read another 256 MB so that the written
+    (dirty) lines are written back before the next timed region starts."""
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
-    w = li.workload(args.workload)
-    dev = torch.device("cuda", local)
-    peaks = load_peaks()
-    # each rank streams an independent video (weak scaling)
-    w = rank_workload(w, rank)
-    streaming = w.kv_past[0] > 0 or w.B > 1
-    x = li.make_inputs(w)
-    params = lc.SelectParams(top_k=w.top_k, density=w.density, window=w.window,
-                             window_mode=w.window_mode)
-    n_chunks = 3
-    if streaming:
+    def flush_l2():
+        flush.zero_()
+        flush_rd.sum()
+    return flush_l2
+
+
+def allowed_pairs(w, cache) -> int:
+    """Number of (query block, key block) pairs the coarse map scores: causal
+    candidates inside the query block's window (all of them without one)."""
+    nQT = (w.q_frames + 1) // 2
+
+    def axis_sizes(n):
+        out = []
+        for i in range(n):
+            if w.window <= 0:
+                lo, hi = 0, n
+            elif w.window_mode >= 2:      # token windows: blocks seen by some token of block i
+                def tw(t, ntok):
+                    s0 = t - w.window // 2
+                    if w.window_mode == 2:
+                        return max(s0, 0), min(s0 + w.window, ntok)
+                    st = max(min(s0, ntok - w.window), 0)
+                    return st, min(st + w.window, ntok)
+                a, _ = tw(8 * i, 8 * n)
+                _, d = tw(8 * i + 7, 8 * n)
+                lo, hi = a // 8, (d - 1) // 8 + 1
+            elif w.window_mode == 0:
+                r = w.window // 2
+                lo, hi = max(i - r, 0), min(i + r + 1, n)
+            else:
+                r = w.window // 2
+                lo = max(min(i - r, n - w.window), 0)
+                hi = min(lo + w.window, n)
+            out.append(hi - lo)
+        return out
+    area = sum(a * b for a in axis_sizes(w.Hb) for b in axis_sizes(w.Wb))
+    total = 0
+    for b in range(w.B):
+        nKT = cache.end(b) // 2 - cache.begin(b) // 2
+        for tq in range(nQT):
+            total += (nKT - nQT + tq + 1) * area
+    return total * w.H
+
+
+def setup_workload(lc, w, x, dev, n_chunks=3):
+    """Device state of one workload and the functions that run one step of it.
+
+    Streaming workloads: a ring cache holding each stream's past frames, then
+    per step lcsa_ingest_chunk (Q pooled, K pooled while K and V are written
+    into the ring), lcsa_select_blocks and lcsa_sparse_attn_fwd, on distinct
+    chunks cycled through the steps. Whole clip: Q, K, V of all 26 frames
+    resident, per step lcsa_pool_qk (Q and K), select and attention."""
+    params = lc.SelectParams(top_k=w.top_k, density=w.density, window=w.window, window_mode=w.window_mode)
+    st = type("Setup", (), {})()
+    st.w = w
+    st.streaming = w.kv_past[0] > 0 or w.B > 1
+    tok_window = w.window if w.window_mode >= li.WINDOW_TRUNCATE_TOKENS else 0
+    if st.streaming:
         cache = lc.KVCache(w.B, w.H, w.cap_frames, w.Y, w.X, w.D, device=dev)
         for b in range(w.B):
             kp = x["k"][b][:, :w.kv_past[b]].unsqueeze(0).to(dev)
             vp = x["v"][b][:, :w.kv_past[b]].unsqueeze(0).to(dev)
             lc.kv_append(cache, kp, vp, lc.pool_qk(kp)[0], stream_offset=b)
-        # distinct chunks cycled through the steps (the stream keeps advancing)
         g = torch.Generator().manual_seed(w.seed + 7)
         shp = (w.B, w.H, w.q_frames, w.Y, w.X, w.D)
         chunks = [(x["q"].to(dev),
                    torch.stack([x["k"][b][:, -w.q_frames:] for b in range(w.B)]).to(dev),
                    torch.stack([x["v"][b][:, -w.q_frames:] for b in range(w.B)]).to(dev))]
         for _ in range(n_chunks - 1):
-            chunks.append(tuple(torch.randn(shp, generator=g).to(torch.bfloat16).to(dev)
-                                for _ in range(3)))
+            chunks.append(tuple(torch.randn(shp, generator=g).to(torch.bfloat16).to(dev) for _ in range(3)))
         step = lc.StreamingStep(cache, w.q_frames, params)
         base_state = cache.state()
-        tok_window = w.window if w.window_mode >= li.WINDOW_TRUNCATE_TOKENS else 0
 
-        def run_step(i, q=None, k=None, v=None, ev=None):
-            if q is None:
-                q, k, v = chunks[i % n_chunks]
+        def run_step(i, ev=None):
+            q, k, v = chunks[i % n_chunks]
             # every step sees the workload's cache lengths (host-side state only);
-            # the append still writes 2 frames and the pooled K into the ring
+            # the append still writes the chunk's frames and pooled K into the ring
             step.cache.set_state(base_state)
             if ev is not None:
                 ev[0].record()
-            lc.pool_qk(q, None, step.q_pool)
+            lc.ingest_chunk(q, step.cache, k, v, step.q_pool)
             if ev is not None:
                 ev[1].record()
-            lc.kv_append(step.cache, k, v)  # pools K while copying it
-            if ev is not None:
-                ev[2].record()
             lc.select_blocks(step.q_pool, step.q_frames, step.cache, step.params, step.kmax,
                              step.blk_idx, step.blk_cnt, step.workspace)
             if ev is not None:
-                ev[3].record()
-            lc.sparse_attn_fwd(q, step.cache, step.blk_idx, step.blk_cnt, step.o, step.lse, workspace=step.attn_ws,
-                               window=tok_window, window_mode=w.window_mode)
+                ev[2].record()
+            lc.sparse_attn_fwd(q, step.cache, step.blk_idx, step.blk_cnt, step.o, step.lse,
+                               workspace=step.attn_ws, window=tok_window, window_mode=w.window_mode)
             if ev is not None:
-                ev[4].record()
+                ev[3].record()
             return step.o
 
-        kernels = ["pool", "kv_append", "select", "attn"]
-        q_frames_step = w.q_frames
-        sel_ref = step
+        def run_split(i, ev):
+            # the ingest as two launches: Q pooling alone, then the K/V append
+            q, k, v = chunks[i % n_chunks]
+            step.cache.set_state(base_state)
+            ev[0].record()
+            lc.pool_qk(q, None, step.q_pool)
+            ev[1].record()
+            lc.kv_append(step.cache, k, v)
+            ev[2].record()
+
+        def graph_step():
+            step.cache.set_state(base_state)
+            step.graph_step()
+
+        st.kernels = ["ingest", "select", "attn"]
+        st.split_kernels = ["pool", "kv_append"]
+        st.run_split = run_split
+        st.graph_prepare = lambda: (step.cache.set_state(base_state), step.graph_step(*chunks[0]))
+        st.graph_step = graph_step
+        st.cache, st.step, st.chunks, st.base_state = cache, step, chunks, base_state
+        st.blk_idx, st.blk_cnt, st.o = step.blk_idx, step.blk_cnt, step.o
+        st.kmax = step.kmax
     else:
-        # whole clip: Q, K, V of all frames resident; no append
         q = x["q"].to(dev)
         k = x["k"][0].unsqueeze(0).to(dev)
         v = x["v"][0].unsqueeze(0).to(dev)
@@ -263,17 +325,10 @@ def run_ours(args, world, rank, local):
         blk_cnt = torch.empty((1, w.H, nQB), dtype=torch.int32, device=dev)
         o = torch.empty_like(q)
         lse = torch.empty(q.shape[:5], dtype=torch.float32, device=dev)
-        sel_ws = torch.empty(max(lc.select_workspace_bytes(cache, w.q_frames), 16), dtype=torch.uint8,
-                             device=dev)
+        sel_ws = torch.empty(max(lc.select_workspace_bytes(cache, w.q_frames), 16), dtype=torch.uint8, device=dev)
         attn_ws = lc.attn_workspace(w.D, dev)
-        base_state = cache.state()
 
-        class _S:
-            pass
-        sel_ref = _S()
-        sel_ref.blk_idx, sel_ref.blk_cnt, sel_ref.o = blk_idx, blk_cnt, o
-
-        def run_step(i, qq=None, kk=None, vv=None, ev=None):
+        def run_step(i, ev=None):
             if ev is not None:
                 ev[0].record()
             lc.pool_qk(q, k, q_pool, k_pool)
@@ -287,99 +342,186 @@ def run_ours(args, world, rank, local):
                 ev[3].record()
             return o
 
-        kernels = ["pool", "select", "attn"]
-        q_frames_step = w.q_frames
+        st.kernels = ["pool", "select", "attn"]
+        st.split_kernels = []
+        st.graph_step = None
+        st.cache, st.q, st.k, st.v = cache, q, k, v
+        st.blk_idx, st.blk_cnt, st.o = blk_idx, blk_cnt, o
+        st.kmax = kmax
+    st.run_step = run_step
+    return st
 
-    # L2 flush: write 512 MB, then read another 256 MB so that the written
-    # (dirty) lines are written back before the timed step starts
-    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-    flush_rd = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
-    def flush_l2():
-        flush.zero_()
-        flush_rd.sum()
-
-    for i in range(args.warmup):
+def time_events(n, nev, body, flush_l2):
+    """n timed repetitions of body(i, ev) with L2 flushed before each (outside
+    the events); returns the per-repetition lists of event-pair durations."""
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(n)]
+    for i in range(n):
         flush_l2()
-        run_step(i)
+        body(i, evs[i])
+    torch.cuda.synchronize()
+    return [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nev - 1)] for i in range(n)]
+
+
+def measure(lc, st, steps, warmup, flush_l2, peaks, world, clocks=None):
+    """Per-kernel split (eager, CUDA events between the kernels), the
+    whole-step graph replay, and the derived rooflines of one workload."""
+    w = st.w
+    for i in range(warmup):
+        flush_l2()
+        st.run_step(i)
     torch.cuda.synchronize()
     if lc.last_device_error() != 0:
-        raise RuntimeError("device error during warm-up")
-
-    nev = len(kernels) + 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
-    clocks = ClockSampler(local)
+        raise RuntimeError("device error during warm-up (%s)" % w.name)
     barrier(world)
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
+    if clocks is not None:
+        clocks.start()
+        time.sleep(0.3)
     t_wall = time.perf_counter()
-    for i in range(args.steps):
-        flush_l2()
-        run_step(args.warmup + i, ev=evs[i])
+    eager = time_events(steps, len(st.kernels) + 1, lambda i, ev: st.run_step(warmup + i, ev), flush_l2)
+    split = (time_events(steps, len(st.split_kernels) + 1, st.run_split, flush_l2)
+             if st.split_kernels else None)
+    graph_ms = None
+    if st.graph_step is not None:
+        st.graph_prepare()
+        for _ in range(warmup):
+            flush_l2()
+            st.graph_step()
+        g = time_events(steps, 2, lambda i, ev: (ev[0].record(), st.graph_step(), ev[1].record()), flush_l2)
+        graph_ms = statistics.mean(r[0] for r in g)
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall
     barrier(world)
-    time.sleep(0.2)
-    clk = clocks.stop()
+    clk = None
+    if clocks is not None:
+        time.sleep(0.2)
+        clk = clocks.stop()
     if lc.last_device_error() != 0:
-        raise RuntimeError("device error during the timed steps")
-    step_ms = [evs[i][0].elapsed_time(evs[i][-1]) for i in range(args.steps)]
-    per_kernel = {kname: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
-                  for j, kname in enumerate(kernels)}
-    mean_step = statistics.mean(step_ms)
-    mean_step_max = max_over_ranks(mean_step, world)
+        raise RuntimeError("device error during the timed steps (%s)" % w.name)
+
+    per_kernel = {k: statistics.mean(r[j] for r in eager) for j, k in enumerate(st.kernels)}
+    if split is not None:
+        per_kernel.update({k: statistics.mean(r[j] for r in split) for j, k in enumerate(st.split_kernels)})
+    eager_ms = max_over_ranks(statistics.mean(sum(r) for r in eager), world)
+    chunks_per_step = CHUNKS_PER_STEP.get(w.name, 1) * w.B
+    res = {"eager_ms_per_chunk": whole_job_ms_per_chunk(eager_ms, chunks_per_step, world),
+           "graph_ms_per_chunk": (whole_job_ms_per_chunk(max_over_ranks(graph_ms, world), chunks_per_step, world)
+                                  if graph_ms is not None else None),
+           "per_kernel_ms": per_kernel, "clocks": clk, "wall_s_timed": t_wall}
+
+    # attention: algorithmic FLOPs of the kept blocks, tensor-bound
+    flops = attn_flops(st.blk_cnt, st.blk_idx, st.cache, w.Hb, w.Wb, w.D)
+    tflops = flops / (per_kernel["attn"] / 1e3) / 1e12
+    res["attn"] = {"flops": flops, "tflops": tflops, "frac": tflops / peaks["bf16_tflops"]}
+
+    # HBM-side launches: algorithmic bytes per launch
+    tokens_q = w.B * w.H * w.q_frames * w.Y * w.X
+    pooled_row = w.D * 8
+    hbm = {}
+    if st.streaming:
+        tokens_kv = tokens_q                                  # the chunk's new K / V frames
+        bytes_pool = tokens_q * w.D * 2 + (tokens_q // 128) * pooled_row
+        bytes_app = 2 * (2 * tokens_kv * w.D * 2) + (tokens_kv // 128) * pooled_row
+        hbm["pool_gbs"] = bytes_pool / (per_kernel["pool"] / 1e3) / 1e9
+        hbm["kv_append_gbs"] = bytes_app / (per_kernel["kv_append"] / 1e3) / 1e9
+        hbm["ingest_gbs"] = (bytes_pool + bytes_app) / (per_kernel["ingest"] / 1e3) / 1e9
+        res["bytes"] = {"pool": bytes_pool, "kv_append": bytes_app, "ingest": bytes_pool + bytes_app}
+    else:
+        bytes_pool = 2 * tokens_q * w.D * 2 + 2 * (tokens_q // 128) * pooled_row
+        hbm["pool_gbs"] = bytes_pool / (per_kernel["pool"] / 1e3) / 1e9
+        res["bytes"] = {"pool": bytes_pool}
+    res["hbm"] = {k: v / peaks["hbm_gbs"] for k, v in hbm.items()}
+    res["hbm_gbs"] = hbm
+
+    # selection: bytes it must move (pooled Q and the candidates' pooled K in,
+    # block lists out) and its float64 work (one multiply and one add per
+    # channel of every scored pair)
+    rows = w.B * w.H * ((w.q_frames + 1) // 2) * w.Hb * w.Wb
+    n_kblocks = sum((st.cache.end(b) // 2 - st.cache.begin(b) // 2) for b in range(w.B)) * w.Hb * w.Wb * w.H
+    sel_bytes = rows * pooled_row + n_kblocks * pooled_row + rows * st.kmax * 4 + rows * 4
+    pairs = allowed_pairs(w, st.cache)
+    sel_s = per_kernel["select"] / 1e3
+    fp64_tflops = 2.0 * w.D * pairs / sel_s / 1e12
+    q_pool_bytes = rows * pooled_row + (tokens_q * w.D * 2)            # the Q pooling launch
+    pool_ms = per_kernel["pool"]
+    res["select"] = {
+        "ms": per_kernel["select"], "bytes": sel_bytes, "gbs": sel_bytes / sel_s / 1e9,
+        "hbm_frac": sel_bytes / sel_s / 1e9 / peaks["hbm_gbs"],
+        "scored_pairs": pairs, "fp64_tflops": fp64_tflops, "fp64_frac": fp64_tflops / FP64_PEAK_TFLOPS,
+        "pool_plus_select_gbs": (q_pool_bytes + sel_bytes) / ((pool_ms + per_kernel["select"]) / 1e3) / 1e9,
+    }
+    res["select"]["pool_plus_select_hbm_frac"] = res["select"]["pool_plus_select_gbs"] / peaks["hbm_gbs"]
+    return res
+
+
+# float64 peak for the selection's roofline: 148 SMs x 64 FP64 lanes x 2 FLOP
+# (a fused multiply-add) x 1965 MHz (the B200's maximum SM clock); the score
+# kernel issues a separate multiply and add per channel, so its instruction
+# peak is the same 18.6 T instructions/s counted as 2 FLOP each.
+FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
+
+
+EXTRA_WORKLOADS = ["multistream", "uhr_truncate", "uhr_preserve", "uhr_truncate_tok", "uhr_preserve_tok",
+                   "clip_5", "clip", "clip_30"]
+
+
+def run_ours(args, world, rank, local):
+    import block_sparse_causal_lcsa_b200 as lc
+
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    # each rank streams an independent video (weak scaling)
+    w = rank_workload(li.workload(args.workload), rank)
+    x = li.make_inputs(w)
+    st = setup_workload(lc, w, x, dev)
+    flush_l2 = make_flusher(dev)
+    clocks = ClockSampler(local)
+    m = measure(lc, st, args.steps, args.warmup, flush_l2, peaks, world, clocks=clocks)
     chunks_per_step = CHUNKS_PER_STEP.get(args.workload, 1) * w.B
-    value = whole_job_ms_per_chunk(mean_step_max, chunks_per_step, world)
+    per_kernel = m["per_kernel_ms"]
 
-    flops = attn_flops(sel_ref.blk_cnt, sel_ref.blk_idx, cache, w.Hb, w.Wb, w.D)
-    attn_s = per_kernel["attn"] / 1e3
-    achieved_tflops = flops / attn_s / 1e12
-    peak = peaks["bf16_tflops"]
-
-    # e2e: the same step through the API with inputs from pinned host memory and
-    # the output read back, copies inside the timed region
+    # e2e: the same step through the API with the chunk's inputs coming from
+    # pinned host memory and O going back there, copies inside the timed region
     e2e = None
-    if streaming:
-        # chunks from pinned host memory through lc.HostPipeline: each chunk's
+    if st.streaming:
+        # distinct pinned host chunks through lc.HostPipeline: each chunk's
         # inputs cross PCIe while the previous chunk computes, and its O comes
         # back on a third stream; the timed region runs from the first timed
-        # chunk's host-to-device copy to the last chunk's device-to-host copy
-        hq = chunks[0][0].cpu().pin_memory()
-        hk = chunks[0][1].cpu().pin_memory()
-        hv = chunks[0][2].cpu().pin_memory()
-        ho = torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory()
-        pipe = lc.HostPipeline(step)
+        # chunk's host-to-device copy to the last chunk's device-to-host copy.
+        # No L2 flush in this loop: every step's inputs arrive by a fresh copy
+        # and its working set (cache + chunk) is larger than L2.
+        host = [tuple(t.cpu().pin_memory() for t in c) for c in st.chunks]
+        ho = torch.empty(host[0][0].shape, dtype=torch.bfloat16).pin_memory()
+        pipe = lc.HostPipeline(st.step)
         e_start = torch.cuda.Event(enable_timing=True)
         done = None
         for i in range(args.warmup + args.steps):
             if i == args.warmup:
                 torch.cuda.synchronize()
                 e_start.record(pipe.h2d_stream)
-            flush_l2()
-            step.cache.set_state(base_state)
-            done = pipe.submit(hq, hk, hv, ho)
+            st.step.cache.set_state(st.base_state)
+            done = pipe.submit(*host[i % len(host)], ho)
         torch.cuda.synchronize()
-        e2e_ms = e_start.elapsed_time(done) / args.steps
-        e2e_ms = max_over_ranks(e2e_ms, world)
+        e2e_ms = max_over_ranks(e_start.elapsed_time(done) / args.steps, world)
+        hq, hk, hv = host[0]
         e2e = {"value": whole_job_ms_per_chunk(e2e_ms, chunks_per_step, world), "unit": UNIT,
                "h2d_bytes_per_step": hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2,
                "d2h_bytes_per_step": ho.numel() * 2,
-               "pipelined": "copies of chunk i+1 overlap the compute of chunk i (lc.HostPipeline)"}
+               "pipelined": "copies of chunk i+1 overlap the compute of chunk i (lc.HostPipeline); "
+                            "%d distinct host chunks cycled; no L2 flush (inputs arrive by copy)" % len(host)}
     else:
-        hq = q.cpu().pin_memory()
-        hk = k.cpu().pin_memory()
-        hv = v.cpu().pin_memory()
+        hq, hk, hv = st.q.cpu().pin_memory(), st.k.cpu().pin_memory(), st.v.cpu().pin_memory()
         ho = torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory()
         e_start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         e_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         for i in range(args.warmup + args.steps):
             if i >= args.warmup:
                 e_start[i - args.warmup].record()
-            q.copy_(hq, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
-            out = run_step(i)
+            st.q.copy_(hq, non_blocking=True)
+            st.k.copy_(hk, non_blocking=True)
+            st.v.copy_(hv, non_blocking=True)
+            out = st.run_step(i)
             ho.copy_(out, non_blocking=True)
             if i >= args.warmup:
                 e_end[i - args.warmup].record()
@@ -391,43 +533,6 @@ def run_ours(args, world, rank, local):
     if lc.last_device_error() != 0:
         raise RuntimeError("device error during the end-to-end steps")
 
-    # the same step replayed from a CUDA graph (one launch per step), inputs in
-    # the graph's static buffers, L2 flushed outside the timed events
-    graph = None
-    if streaming:
-        step.cache.set_state(base_state)
-        step.graph_step(*chunks[0])
-        g_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        for i in range(args.warmup + args.steps):
-            flush_l2()
-            step.cache.set_state(base_state)
-            if i >= args.warmup:
-                g_ev[i - args.warmup][0].record()
-            step.graph_step()
-            if i >= args.warmup:
-                g_ev[i - args.warmup][1].record()
-        torch.cuda.synchronize()
-        if lc.last_device_error() != 0:
-            raise RuntimeError("device error during the graph steps")
-        g_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in g_ev), world)
-        graph = {"ms_per_chunk": round(whole_job_ms_per_chunk(g_ms, chunks_per_step, world), 4),
-                 "graph_launches_per_step": 1}
-
-    # HBM-side kernels: algorithmic bytes per launch
-    tokens_q = w.B * w.H * q_frames_step * w.Y * w.X
-    if "kv_append" in per_kernel:
-        # pool reads Q (bf16) once and writes one float64 row per block; the
-        # append reads the new K and V once, writes them into the ring and
-        # writes K's pooled rows
-        bytes_pool = tokens_q * w.D * 2 + (tokens_q // 128) * w.D * 8
-        bytes_app = 2 * (2 * tokens_q * w.D * 2) + (tokens_q // 128) * w.D * 8
-        hbm = {"pool_gbs": bytes_pool / (per_kernel["pool"] / 1e3) / 1e9,
-               "kv_append_gbs": bytes_app / (per_kernel["kv_append"] / 1e3) / 1e9}
-    else:
-        # whole clip: pool reads Q and K once and writes their pooled rows
-        bytes_pool = 2 * tokens_q * w.D * 2 + 2 * (tokens_q // 128) * w.D * 8
-        hbm = {"pool_gbs": bytes_pool / (per_kernel["pool"] / 1e3) / 1e9}
-
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "attn_fwd_%s.traffic.txt" % args.workload)
     if os.path.exists(tfile):
@@ -435,8 +540,8 @@ def run_ours(args, world, rank, local):
         if rec.get("source_hash", "").strip() == attn_source_hash():
             traffic = int(rec["bytes_per_launch"])
 
-    # kernels per timed step: the ingest (streaming graph: Q pooling and the
-    # fused K/V append in one launch; clip: Q and K pooling), score + top-K, the
+    # kernels per timed step of the headline (graph replay): the ingest
+    # (streaming: one fused launch; clip: Q and K pooling), score + top-K, the
     # attention and, when its last wave is split, the merge of the halves
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     units = w.B * w.H * ((w.q_frames + 1) // 2) * w.Hb * w.Wb
@@ -445,15 +550,15 @@ def run_ours(args, world, rank, local):
     # the headline is the step as a user runs it in production: replayed from a
     # CUDA graph (same kernels, same work, one launch); the eager run with CUDA
     # events between the kernels gives the per-kernel split
-    eager_value = value
-    step_ms = mean_step_max
-    if graph is not None:
-        value = graph["ms_per_chunk"]
-        step_ms = value * chunks_per_step * world
+    value = m["graph_ms_per_chunk"] if m["graph_ms_per_chunk"] is not None else m["eager_ms_per_chunk"]
+    step_ms = value * chunks_per_step * world
+    peak = peaks["bf16_tflops"]
+    clk = m["clocks"]
+    sm_mhz = (clk or {}).get("sm_mhz") or peaks.get("sm_max_mhz") or 1965.0
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
-        "eager_ms_per_chunk": round(eager_value, 4),
+        "eager_ms_per_chunk": round(m["eager_ms_per_chunk"], 4),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16, shapes of the pages' 768x1408 workload)",
         "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload,
@@ -464,22 +569,65 @@ def run_ours(args, world, rank, local):
                    "select_precision": "fp64 scores, exact top-K",
                    "parallelism": "independent stream per GPU" if world > 1 else "single GPU"},
         "per_kernel_ms": {k2: round(v2, 5) for k2, v2 in per_kernel.items()},
-        "sparse_attn_tflops": round(achieved_tflops, 2),
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd", "achieved": round(achieved_tflops, 2),
-                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved_tflops / peak, 4),
+        "sparse_attn_tflops": round(m["attn"]["tflops"], 2),
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd", "achieved": round(m["attn"]["tflops"], 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(m["attn"]["tflops"] / peak, 4),
                      "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % peaks["source"],
-                     "flops_per_launch": flops, "traffic": traffic},
-        "hbm_kernels": {k2: round(v2, 1) for k2, v2 in hbm.items()},
-        "cuda_graph": graph,
+                     "flops_per_launch": m["attn"]["flops"], "traffic": traffic,
+                     # the same FLOPs against the dense bf16 tensor peak at the SM clock
+                     # sampled during the run (8192 FLOP per clock per SM x 148 SMs)
+                     "frac_of_clock_peak": round(m["attn"]["tflops"] / (148 * 8192 * sm_mhz * 1e6 / 1e12), 4),
+                     "clock_peak_tflops": round(148 * 8192 * sm_mhz * 1e6 / 1e12, 1)},
+        "hbm_kernels": {k2: round(v2, 1) for k2, v2 in m["hbm_gbs"].items()},
+        "hbm_frac": {k2: round(v2, 4) for k2, v2 in m["hbm"].items()},
+        "select": {k2: (round(v2, 5) if isinstance(v2, float) else v2) for k2, v2 in m["select"].items()},
+        "select_fp64_peak": "%.1f TFLOP/s = 148 SMs x 64 FP64 lanes x 2 FLOP x 1965 MHz (nominal)" % FP64_PEAK_TFLOPS,
+        "cuda_graph": ({"ms_per_chunk": round(m["graph_ms_per_chunk"], 4), "graph_launches_per_step": 1}
+                       if m["graph_ms_per_chunk"] is not None else None),
         "hbm_peak_gbs": peaks["hbm_gbs"],
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
-        "wall_s_timed": round(t_wall, 4),
+        "wall_s_timed": round(m["wall_s_timed"], 4),
     }
+    del st
+    torch.cuda.empty_cache()
+    if not args.no_workloads and world == 1:
+        line["workloads"] = extra_workloads(lc, dev, peaks, args, flush_l2)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, x, budget_s=args.cpu_budget)
     return line
+
+
+def extra_workloads(lc, dev, peaks, args, flush_l2):
+    """The other configurations of the metric, a few steps each: ms per chunk
+    (graph replay for streams, eager for the whole clip, divided by its 13
+    chunks), attention TFLOP/s and fraction of the bf16 peak, selection."""
+    out = {}
+    cache_inputs = {}
+    for name in EXTRA_WORKLOADS:
+        w = li.workload(name)
+        key = (w.seed, w.structure, w.B, w.Y, w.X, w.q_frames, w.kv_past)
+        if key not in cache_inputs:
+            cache_inputs.clear()
+            cache_inputs[key] = li.make_inputs(w)
+        x = cache_inputs[key]
+        st = setup_workload(lc, w, x, dev)
+        m = measure(lc, st, args.extra_steps, 3, flush_l2, peaks, 1)
+        out[name] = {
+            "ms_per_chunk": round(m["graph_ms_per_chunk"] if m["graph_ms_per_chunk"] is not None
+                                  else m["eager_ms_per_chunk"], 4),
+            "timed_as": "graph replay" if m["graph_ms_per_chunk"] is not None else "eager, clip / 13 chunks",
+            "attn_ms": round(m["per_kernel_ms"]["attn"], 4),
+            "attn_tflops": round(m["attn"]["tflops"], 1), "attn_frac": round(m["attn"]["frac"], 4),
+            "select_ms": round(m["select"]["ms"], 4), "select_fp64_frac": round(m["select"]["fp64_frac"], 4),
+            "pool_gbs": round(m["hbm_gbs"]["pool_gbs"], 1),
+            "ingest_gbs": round(m["hbm_gbs"].get("ingest_gbs", float("nan")), 1) if st.streaming else None,
+            "kept_pairs": int(st.blk_cnt.sum().item()),
+        }
+        del st, m
+        torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------------------- oracle arm
@@ -557,6 +705,7 @@ def run_backward(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import lcsa_oracle as orc
         t0 = time.perf_counter()
+        c0 = time.process_time()
         h = 0
         qh, kh, vh = orc.widen(x["q"][0, h]), orc.widen(x["k"][0][h]), orc.widen(x["v"][0][h])
         sel = [idx[0, h, i, :int(cnt[0, h, i])].cpu().numpy() for i in range(cnt.shape[2])]
@@ -574,9 +723,11 @@ def run_backward(args, world, rank, local):
             if time.perf_counter() - t0 > args.cpu_budget:
                 break
         el = time.perf_counter() - t0
+        cpu_used = time.process_time() - c0
         total_kept = int(cnt.sum().item())
         cpu_ms = el / kept * total_kept * 1e3
-        line["cpu_baseline"] = {"value": round(cpu_ms, 1), "unit": "ms/clip", "cores": _threads(), "kind": "oracle",
+        line["cpu_baseline"] = {"value": round(cpu_ms, 1), "unit": "ms/clip", "cores": round(cpu_used / el, 2),
+                                "cpu_model": cpu_model(), "kind": "oracle",
                                 "sample": "%d query blocks (%d kept block pairs) of head 0, attend_rows_backward "
                                           "in fp64, scaled by kept pairs to all %d" % (n_rows, kept, total_kept)}
     return line
@@ -672,25 +823,54 @@ def _threads():
         return os.cpu_count()
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+class CpuMeter:
+    """Wall time and the process's CPU time over a region: their ratio is the
+    number of cores the oracle actually kept busy (its per-block loops are
+    mostly single-threaded numpy; only the products use several BLAS threads)."""
+
+    def __enter__(self):
+        self.w0, self.c0 = time.perf_counter(), time.process_time()
+        return self
+
+    def __exit__(self, *exc):
+        self.wall = time.perf_counter() - self.w0
+        self.cpu = time.process_time() - self.c0
+
+    @property
+    def cores(self) -> float:
+        return round(self.cpu / self.wall, 2) if self.wall > 0 else 1.0
+
+
 def cpu_baseline(w, x, budget_s=15.0):
     """The fp64 oracle as it stands, on whole heads of the workload until the
     budget is spent; scaled to ms per chunk."""
     from oracle import lcsa_oracle as orc
 
-    t0 = time.perf_counter()
     done = 0
     streams = [(b, h) for b in range(w.B) for h in range(w.H)]
-    for b, h in streams:
-        orc.lcsa_head(orc.widen(x["q"][b, h]), orc.widen(x["k"][b][h]), orc.widen(x["v"][b][h]),
-                      top_k=w.top_k, density=w.density, window=w.window, mode=w.window_mode)
-        done += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    el = time.perf_counter() - t0
-    per_chunk_ms = el / done * len(streams) / (CHUNKS_PER_STEP.get(w.name, 1) * w.B) * 1e3
-    return {"value": round(per_chunk_ms, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+    with CpuMeter() as meter:
+        for b, h in streams:
+            orc.lcsa_head(orc.widen(x["q"][b, h]), orc.widen(x["k"][b][h]), orc.widen(x["v"][b][h]),
+                          top_k=w.top_k, density=w.density, window=w.window, mode=w.window_mode)
+            done += 1
+            if time.perf_counter() - meter.w0 > budget_s:
+                break
+    per_chunk_ms = meter.wall / done * len(streams) / (CHUNKS_PER_STEP.get(w.name, 1) * w.B) * 1e3
+    return {"value": round(per_chunk_ms, 2), "unit": UNIT, "cores": meter.cores, "kind": "oracle",
+            "threads_available": _threads(), "cpu_model": cpu_model(),
             "sample": "%d of %d (stream, head) units of the workload, whole path (pool, select, "
-                      "attention) in fp64, scaled to the full chunk" % (done, len(streams))}
+                      "attention) in fp64, scaled to the full chunk; cores = process CPU time / wall "
+                      "time" % (done, len(streams))}
 
 
 def run_reference(args, world, rank):
@@ -702,23 +882,26 @@ def run_reference(args, world, rank):
 
     units = [(b, h) for b in range(w.B) for h in range(w.H)]
     times = []
+    cpu = 0.0
     for i in range(args.warmup + args.steps):
         b, h = units[i % len(units)]
-        t0 = time.perf_counter()
-        orc.lcsa_head(orc.widen(x["q"][b, h]), orc.widen(x["k"][b][h]), orc.widen(x["v"][b][h]),
-                      top_k=w.top_k, density=w.density, window=w.window, mode=w.window_mode)
+        with CpuMeter() as meter:
+            orc.lcsa_head(orc.widen(x["q"][b, h]), orc.widen(x["k"][b][h]), orc.widen(x["v"][b][h]),
+                          top_k=w.top_k, density=w.density, window=w.window, mode=w.window_mode)
         if i >= args.warmup:
-            times.append(time.perf_counter() - t0)
+            times.append(meter.wall)
+            cpu += meter.cpu
     per_chunk_ms = statistics.mean(times) * len(units) / (CHUNKS_PER_STEP.get(args.workload, 1) * w.B) * 1e3
     sample = ("one (stream, head) unit per step, whole path (pool, select, attention) in fp64, "
-              "scaled by %d units to the full chunk" % len(units))
+              "scaled by %d units to the full chunk; cores = process CPU time / wall time" % len(units))
     return {
         "impl": "reference", "metric": METRIC, "value": round(per_chunk_ms, 2), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(statistics.mean(times) * 1e3, 2), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload},
-        "cpu_baseline": {"value": round(per_chunk_ms, 2), "unit": UNIT, "cores": _threads(),
+        "cpu_baseline": {"value": round(per_chunk_ms, 2), "unit": UNIT, "cores": round(cpu / sum(times), 2),
+                         "threads_available": _threads(), "cpu_model": cpu_model(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(per_chunk_ms, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -734,6 +917,9 @@ def main():
     ap.add_argument("--workload", default="chunk", choices=sorted(WORKLOAD_TEXT))
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other configurations (multistream, UHR, clip densities) in the headline line")
+    ap.add_argument("--extra-steps", type=int, default=5, help="timed steps per extra configuration")
     ap.add_argument("--mode", default="fwd", choices=["fwd", "bwd", "segment"],
                     help="fwd: the streaming step (default); bwd: the attention backward on a clip; "
                          "segment: stage-1 dense segment attention, forward + backward")
