@@ -9,16 +9,20 @@
 //               (5-D tensor maps over (d, x, y, frame, stream*head); one box =
 //               one frame of a block = 64 tokens x 64 channels, 128-byte
 //               swizzled). A K stage is released as soon as S_j has consumed
-//               it, a V stage once PV_j has; separate producers let the K
-//               loads run ahead of the V stages the softmax holds up.
+//               it (the S_j barrier), a V stage once PV_j has (the PV_j
+//               barrier); separate producers let the K loads run ahead of the
+//               V stages the softmax holds up.
 //   warp 1      MMA issuer (one thread): S_j = Q K_j^T into one of THREE TMEM
 //               score buffers (128 lanes x 128 fp32 columns each), then
-//               O += P_j V_j with P_j read from tensor memory. Scores run up to
-//               two blocks ahead of the softmax (S_{j+2} is issued right after
-//               PV_j), so neither side waits for the other in steady state.
-//               Before an S MMA reuses the buffer a PV MMA read P from, the
-//               issuer waits for that PV to complete: MMAs into different
-//               accumulators are not ordered with respect to each other.
+//               O += P_j V_j with P_j read from tensor memory. Scores run two
+//               blocks ahead of the softmax: S_{j+2} is issued before PV_j, as
+//               soon as PV_{j-1} has completed (it overwrites the buffer P_{j-1}
+//               was read from; MMAs into different accumulators are not ordered
+//               with respect to each other). Issuing S_{j+2} after PV_j
+//               instead put the issue of PV_j on the softmax's critical path.
+//               The PV barriers are one per score buffer: with two (by parity)
+//               and this order, the final wait for PV_{n-1} could match a phase
+//               of PV_{n-3} that had not completed yet.
 //   warps 2-5   softmax warpgroup, one query row per thread (= TMEM lane):
 //               tcgen05.ld of S_j, mask the missing frame of a one-frame
 //               block, running max with lazy rescaling of O (only when the
@@ -45,6 +49,9 @@ namespace lcsa {
 constexpr int K_STAGES = 3;
 constexpr int V_STAGES = 3;
 constexpr int S_BUFS = 3;
+// a K stage is free once the score product that read it has completed, a V
+// stage once its PV has: the stages reuse the score buffers' barriers
+static_assert(K_STAGES == S_BUFS && V_STAGES == S_BUFS, "K/V stages follow the score buffers");
 constexpr int EXP_POLY_EVERY = 1 << 30;   // exponent pairs sent to the FMA-pipe polynomial (none)
 
 template <int D>
@@ -64,13 +71,11 @@ struct AttnLayout {
 enum : int {
   B_Q_FULL = 0,
   B_K_FULL = 1,                        // K_STAGES
-  B_K_EMPTY = B_K_FULL + K_STAGES,     // K_STAGES
-  B_V_FULL = B_K_EMPTY + K_STAGES,     // V_STAGES
-  B_V_EMPTY = B_V_FULL + V_STAGES,     // V_STAGES
-  B_S_FULL = B_V_EMPTY + V_STAGES,     // S_BUFS
+  B_V_FULL = B_K_FULL + K_STAGES,      // V_STAGES
+  B_S_FULL = B_V_FULL + V_STAGES,      // S_BUFS; S_j done also frees K stage j % K_STAGES
   B_P_FULL = B_S_FULL + S_BUFS,        // S_BUFS (128 softmax arrivals)
-  B_PV_DONE = B_P_FULL + S_BUFS,       // 2, by parity of the block index
-  B_DRAIN = B_PV_DONE + 2,
+  B_PV_DONE = B_P_FULL + S_BUFS,       // S_BUFS; PV_j done also frees V stage j % V_STAGES
+  B_DRAIN = B_PV_DONE + S_BUFS,
   B_COUNT = B_DRAIN + 1
 };
 
@@ -246,7 +251,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         int x8, y8, s0, s1;
         tile_coords(blk, x8, y8, s0, s1);
         const int ks = j % K_STAGES;
-        if (j >= K_STAGES && !wait_bounded(bar(B_K_EMPTY + ks), ((j / K_STAGES) - 1) & 1, w)) break;
+        if (j >= K_STAGES && !wait_bounded(bar(B_S_FULL + ks), ((j / K_STAGES) - 1) & 1, w)) break;
         mbar_arrive_expect_tx(bar(B_K_FULL + ks), L::TILE_BYTES);
         load_tile(&tmK, sbase + L::OFF_K + ks * L::TILE_BYTES, bar(B_K_FULL + ks), x8, y8, s0, s1);
         issued_k = j + 1;
@@ -269,7 +274,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         int x8, y8, s0, s1;
         tile_coords(blk, x8, y8, s0, s1);
         const int vs = j % V_STAGES;
-        if (j >= V_STAGES && !wait_bounded(bar(B_V_EMPTY + vs), ((j / V_STAGES) - 1) & 1, w)) break;
+        if (j >= V_STAGES && !wait_bounded(bar(B_PV_DONE + vs), ((j / V_STAGES) - 1) & 1, w)) break;
         mbar_arrive_expect_tx(bar(B_V_FULL + vs), L::TILE_BYTES);
         load_tile(&tmV, sbase + L::OFF_V + vs * L::TILE_BYTES, bar(B_V_FULL + vs), x8, y8, s0, s1);
         issued_v = j + 1;
@@ -298,7 +303,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                   desc_sw128(ka + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(B_S_FULL + j % S_BUFS));
-        umma_commit(bar(B_K_EMPTY + ks));
         return true;
       };
       bool ok = wait_bounded(bar(B_Q_FULL), 0, w);
@@ -308,6 +312,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (ok && n > 1) ok = issue_s(1);
       }
       for (int j = 0; ok && j < n; ++j) {
+        if (j + 2 < n) {
+          // S_{j+2} overwrites the buffer PV_{j-1} read P_{j-1} from. MMAs into
+          // different accumulators are not ordered, so wait until PV_{j-1} has
+          // completed. S_{j+2} goes out ahead of PV_j: it does not need P_j, so
+          // the softmax of block j+2 does not wait for the issue of PV_j.
+          if (j >= 1 && !(ok = wait_bounded(bar(B_PV_DONE + (j - 1) % S_BUFS), ((j - 1) / S_BUFS) & 1, w))) break;
+          if (!(ok = issue_s(j + 2))) break;
+        }
         const int sb = j % S_BUFS;
         const int vs = j % V_STAGES;
         if (!(ok = wait_bounded(bar(B_P_FULL + sb), (j / S_BUFS) & 1, w))) break;
@@ -323,15 +335,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                   desc_sw128(va + kk * 2048, L::CHUNK_BYTES, 1024), ID_PV,
                   (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(bar(B_PV_DONE + (j & 1)));
-        umma_commit(bar(B_V_EMPTY + vs));
-        if (j + 2 < n) {
-          // S_{j+2} overwrites the buffer PV_{j-1} read P_{j-1} from. MMAs into
-          // different accumulators are not ordered, so wait until PV_{j-1}
-          // has completed (normally long done: PV_j was queued behind it).
-          if (j >= 1 && !(ok = wait_bounded(bar(B_PV_DONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, w))) break;
-          if (!(ok = issue_s(j + 2))) break;
-        }
+        umma_commit(bar(B_PV_DONE + sb));
       }
       // no MMA may still be running when the tensor memory is released
       umma_commit(bar(B_DRAIN));
@@ -348,6 +352,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     float m_run = -INFINITY, l_run = 0.f;         // running max (log2 units) and sum
     bool done = n > 0;
     int next_blk = n > 0 ? checked(blist[0]) : 0;
+    int raw_blk = n > 1 ? blist[1] : 0;
     // token-level window of this row's query token (a key token is visible iff
     // its y and x lie in these ranges)
     int wy0 = 0, wy1 = 0, wx0 = 0, wx1 = 0;
@@ -359,7 +364,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const int sb = j % S_BUFS;
       const int blk = next_blk;
       const bool partial = oldest_partial && blk < HbWb;
-      if (j + 1 < n) next_blk = checked(blist[j + 1]);
+      // block j+1's id was loaded one block ago and block j+2's is loaded now:
+      // the load's latency never stalls the row
+      if (j + 1 < n) next_blk = checked(raw_blk);
+      if (j + 2 < n) raw_blk = blist[j + 2];
       if (!warp_wait(bar(B_S_FULL + sb), (j / S_BUFS) & 1, w)) { done = false; break; }
       tc_fence_after();
       uint32_t s[128];
@@ -410,7 +418,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (j == 0 || mx > m_run + 8.f) m_new = mx;
       if (j > 0 && __any_sync(0xffffffffu, m_new != m_run)) {
         // O may only be rescaled once PV_{j-1} has finished
-        if (!warp_wait(bar(B_PV_DONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, w)) { done = false; break; }
+        if (!warp_wait(bar(B_PV_DONE + (j - 1) % S_BUFS), ((j - 1) / S_BUFS) & 1, w)) { done = false; break; }
         tc_fence_after();
         // 1 for rows whose max did not change (also rows still at -inf, where the difference is NaN)
         const float alpha = m_new == m_run ? 1.f : ex2_approx(m_run - m_new);
@@ -462,7 +470,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tc_fence_before();
       mbar_arrive(bar(B_P_FULL + sb));
     }
-    if (done) done = warp_wait(bar(B_PV_DONE + ((n - 1) & 1)), ((n - 1) >> 1) & 1, w);
+    if (done) done = warp_wait(bar(B_PV_DONE + (n - 1) % S_BUFS), ((n - 1) / S_BUFS) & 1, w);
     const bool row_valid = !(fq0 < 0 && r < 64);
     const int f = r >> 6, yy = (r >> 3) & 7, xx = r & 7;
     const int frame = fq0 + f;
