@@ -28,9 +28,9 @@
 //               block, running max with lazy rescaling of O (only when the
 //               max grows by more than 2^8), P = 2^(s*log2e/sqrt(d) - m) with
 //               packed fp32x2 arithmetic - exponentials on the
-//               special-function unit (every EXP_POLY_EVERY-th pair could go
-//               to a polynomial on the FMA pipe; measured slower here, so
-//               none does) - rounded to bf16 with integer ops
+//               special-function unit (sending some of them to a polynomial
+//               on the FMA pipe measured slower here) - rounded to bf16 with
+//               integer ops
 //               (the special-function pipe also runs float->bf16
 //               conversions, so they would compete with the exponentials) and
 //               stored with tcgen05.st over the first 64 columns of S_j's
@@ -52,7 +52,6 @@ constexpr int S_BUFS = 3;
 // a K stage is free once the score product that read it has completed, a V
 // stage once its PV has: the stages reuse the score buffers' barriers
 static_assert(K_STAGES == S_BUFS && V_STAGES == S_BUFS, "K/V stages follow the score buffers");
-constexpr int EXP_POLY_EVERY = 1 << 30;   // exponent pairs sent to the FMA-pipe polynomial (none)
 
 template <int D>
 struct AttnLayout {
@@ -443,14 +442,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sc2, nm2);
-        uint64_t e2;
-        if ((c % EXP_POLY_EVERY) == EXP_POLY_EVERY - 1) {
-          e2 = exp2_poly_f2(x2);
-        } else {
-          float x0, x1;
-          f2_unpack(x2, x0, x1);
-          e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
-        }
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        const uint64_t e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
         if (c & 1) acc1 = f2_add(acc1, e2);
         else acc0 = f2_add(acc0, e2);
         float e0, e1;

@@ -158,7 +158,7 @@ __global__ void stalled_wait_kernel(uint64_t limit_ns, unsigned int* err) {
   }
 }
 
-// Evaluates the attention kernel's FMA-pipe 2^x polynomial elementwise.
+// Evaluates the FMA-pipe 2^x polynomial (exp2_poly_f2) elementwise.
 __global__ void exp2_poly_kernel(const float* x, float* y, int64_t n) {
   const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
   if (i + 1 < n) {

@@ -442,10 +442,11 @@ LCSA_API lcsa_status lcsa_debug_stalled_wait(uint64_t limit_ns, lcsa_stream_t st
 
 /*
  * Test hook: y[i] = 2^x[i] (x[i] <= 8) evaluated with the FMA-pipe
- * polynomial that the attention softmax can use in place of the
- * special-function unit for part of its exponentials (range reduction
- * x = n + f, |f| <= 1/2, degree-3 minimax polynomial for 2^f, exponent add
- * for 2^n). x, y: device float32 arrays of n elements.
+ * polynomial that was measured as a stand-in for part of the attention
+ * softmax's special-function-unit exponentials (slower there; the kernel
+ * does not use it): range reduction x = n + f, |f| <= 1/2, degree-3
+ * minimax polynomial for 2^f, exponent add for 2^n. x, y: device float32
+ * arrays of n elements.
  */
 LCSA_API lcsa_status lcsa_debug_exp2_poly(const float* x, float* y, int64_t n,
                                           lcsa_stream_t stream);
