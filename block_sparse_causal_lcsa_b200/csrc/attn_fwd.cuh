@@ -101,6 +101,27 @@ struct AttnParams {
   int64_t kv_end[64];
 };
 
+// Exact n / d and n % d for 0 <= n < 2^22 and d >= 1, from a float
+// reciprocal: n and the quotient are below 2^23, so the truncated product is
+// within one of the quotient and one correction step makes it exact (checked
+// for every n < 2^22 on about a thousand divisors).
+struct SmallDiv {
+  int d;
+  float inv;
+  __device__ explicit SmallDiv(int d_) : d(d_), inv(1.0f / static_cast<float>(d_)) {}
+  __device__ __forceinline__ void divmod(int n, int& q, int& r) const {
+    q = __float2int_rz(__int2float_rn(n) * inv);
+    r = n - q * d;
+    if (r < 0) {
+      --q;
+      r += d;
+    } else if (r >= d) {
+      ++q;
+      r -= d;
+    }
+  }
+};
+
 // Warp-uniform bounded wait: every lane polls, all lanes agree on the result.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
   const bool ok = wait_bounded(bar, parity, w);
@@ -200,15 +221,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
   };
   // Ring slots of a key block's two frames; a one-frame block loads its frame twice.
+  // The host passes frame numbers shifted down by whole multiples of the ring
+  // capacity, so they lie in [0, 2 cap): a ring slot is one conditional
+  // subtract. The divisions use SmallDiv (a few instructions, not a software
+  // integer division): the producers share sub-partitions with softmax warps.
+  const int cap = p.cap;
+  const int begin32 = static_cast<int>(begin), m_first32 = static_cast<int>(m_first);
+  const SmallDiv div_blocks(HbWb), div_row(p.Wb);
   auto tile_coords = [&](int blk, int& x8, int& y8, int& s0, int& s1) {
-    const int tk = blk / HbWb, spk = blk % HbWb;
-    const int64_t m = m_first + tk;
-    const int64_t a1 = 2 * m + 1;
-    const int64_t a0 = (2 * m < begin) ? a1 : 2 * m;
-    s0 = static_cast<int>(a0 % p.cap);
-    s1 = static_cast<int>(a1 % p.cap);
-    x8 = 8 * (spk % p.Wb);
-    y8 = 8 * (spk / p.Wb);
+    int tk, spk, yb, xb;
+    div_blocks.divmod(blk, tk, spk);
+    div_row.divmod(spk, yb, xb);
+    const int a1 = 2 * (m_first32 + tk) + 1;
+    const int a0 = a1 - 1 < begin32 ? a1 : a1 - 1;
+    s0 = a0 >= cap ? a0 - cap : a0;
+    s1 = a1 >= cap ? a1 - cap : a1;
+    x8 = 8 * xb;
+    y8 = 8 * yb;
   };
 
   if (threadIdx.x == 0) {
@@ -292,14 +321,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int ks = j % K_STAGES;
         if (!wait_bounded(bar(B_K_FULL + ks), (j / K_STAGES) & 1, w)) return false;
         tc_fence_after();
-        const uint32_t qa = sbase + L::OFF_Q;
-        const uint32_t ka = sbase + L::OFF_K + ks * L::TILE_BYTES;
+        // one descriptor per operand; a step's is the base plus its byte offset
+        // / 16 (the 14-bit address field: shared addresses stay below 2^18)
+        const uint64_t qd = desc_sw128(sbase + L::OFF_Q, 16, 1024);
+        const uint64_t kd = desc_sw128(sbase + L::OFF_K + ks * L::TILE_BYTES, 16, 1024);
+        const uint32_t sd = tmem + (j % S_BUFS) * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           // K-major operands: 16 channels = 32 bytes inside a 128-byte swizzled row
-          const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + (j % S_BUFS) * 128, desc_sw128(qa + off, 16, 1024),
-                  desc_sw128(ka + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
+          const uint32_t off16 = ((kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32) >> 4;
+          umma_ss(sd, qd + off16, kd + off16, ID_S, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(B_S_FULL + j % S_BUFS));
         return true;
@@ -325,14 +356,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (!(ok = wait_bounded(bar(B_V_FULL + vs), (j / V_STAGES) & 1, w))) break;
         tc_fence_after();
         const uint32_t va = sbase + L::OFF_V + vs * L::TILE_BYTES;
+        const uint64_t vd = desc_sw128(va, L::CHUNK_BYTES, 1024);
+        const uint32_t pa = tmem + sb * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           // A = P (16 keys = 8 packed columns of S_j's TMEM buffer); B = V
           // (MN-major: channels contiguous), 16 keys = 16 rows of 128 bytes,
           // 64-channel columns 16 KB apart.
-          umma_ts(tmem + TMEM_O_COL, tmem + sb * 128 + kk * 8,
-                  desc_sw128(va + kk * 2048, L::CHUNK_BYTES, 1024), ID_PV,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + TMEM_O_COL, pa + kk * 8, vd + kk * (2048 >> 4), ID_PV, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(bar(B_PV_DONE + sb));
       }
@@ -381,8 +412,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       if (p.win > 0) {
         // rows / columns of the key block (8 x 8 tokens, both frames alike) inside the window
-        const int spk = blk % HbWb;
-        const int ry = 8 * (spk / p.Wb), rx = 8 * (spk % p.Wb);
+        int tk, spk, yb, xb;
+        div_blocks.divmod(blk, tk, spk);
+        div_row.divmod(spk, yb, xb);
+        const int ry = 8 * yb, rx = 8 * xb;
         const int ylo = min(max(wy0 - ry, 0), 8), yhi = min(max(wy1 - ry, 0), 8);
         const int xlo = min(max(wx0 - rx, 0), 8), xhi = min(max(wx1 - rx, 0), 8);
         const uint32_t ym = ((1u << yhi) - 1u) & ~((1u << ylo) - 1u);

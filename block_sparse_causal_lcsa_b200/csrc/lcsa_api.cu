@@ -735,6 +735,10 @@ static lcsa_status attn_fwd_impl(const lcsa_tensor* q, const lcsa_kv_cache* kv, 
     return LCSA_ERR_SHAPE;
   for (int b = 0; b < kv->B; ++b)
     if (kv->end[b] - kv->begin[b] < 1) return LCSA_ERR_SHAPE;
+  // key block ids lie below (cap / 2) * Hb * Wb; the kernel splits them with a
+  // float reciprocal (SmallDiv) that is exact below 2^22
+  if (static_cast<int64_t>(kv->cap_frames / 2) * (kv->Y / 8) * (kv->X / 8) >= (int64_t{1} << 22))
+    return LCSA_ERR_SHAPE;
   if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LCSA_ERR_ALIGN;
   int dev;
   unsigned int* err;

@@ -318,6 +318,9 @@ LCSA_API lcsa_status lcsa_select_blocks_noalloc(const double* q_pool, int32_t q_
  * lse      device, float32 contiguous [B][H][Tq][Y][X] natural-log
  *          log-sum-exp of each row's scaled logits, or NULL.
  * bf16 tensor-core products with float32 accumulation and softmax.
+ * LCSA_ERR_SHAPE, before any device work, also when a cache holds 2^22 or
+ * more key blocks ((cap_frames / 2) * (Y / 8) * (X / 8)): the kernel splits
+ * block ids with a float reciprocal that is exact below that.
  */
 LCSA_API lcsa_status lcsa_sparse_attn_fwd(const lcsa_tensor* q, const lcsa_kv_cache* kv,
                                  const int32_t* blk_idx, const int32_t* blk_cnt,

@@ -98,6 +98,23 @@ def test_argument_errors_before_any_launch(lib):
     assert lib.lcsa_select_blocks(0x4000, 2, C.byref(kv), C.byref(sp), 0x5000, 0x6000, 0x7000, 1 << 40, None) == _abi.ERR_SHAPE
 
 
+def test_attention_rejects_caches_of_2_22_key_blocks(lib):
+    """Key block ids are split in the kernel with a float reciprocal that is
+    exact below 2^22: a cache of (cap/2) * Hb * Wb >= 2^22 key blocks is an
+    LCSA_ERR_SHAPE before any device work (the pointers here are never used)."""
+    from block_sparse_causal_lcsa_b200 import _abi
+    t = _abi.Tensor(0x1000, 1, 1, 2, 64, 64, 128, 0, 0, 0, 0, 0)
+    t.stride_x, t.stride_y, t.stride_t = 128, 64 * 128, 64 * 64 * 128
+    t.stride_h = t.stride_b = 2 * t.stride_t
+    kv = _abi.KVCacheStruct()
+    kv.k, kv.v, kv.k_pool = 0x1000, 0x2000, 0x3000
+    kv.B, kv.H, kv.Y, kv.X, kv.D = 1, 1, 64, 64, 128
+    kv.cap_frames = 2 * (1 << 16)                    # 2^16 temporal blocks x 64 spatial = 2^22
+    kv.begin[0], kv.end[0] = 0, 2
+    args = (C.byref(t), C.byref(kv), 0x5000, 0x6000, 1, C.byref(t), None, None)
+    assert lib.lcsa_sparse_attn_fwd(*args) == _abi.ERR_SHAPE
+
+
 def test_select_kmax_host_rule(lib):
     from block_sparse_causal_lcsa_b200 import _abi
     kv = _abi.KVCacheStruct()
