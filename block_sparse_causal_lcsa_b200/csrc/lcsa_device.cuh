@@ -318,15 +318,11 @@ __device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t x) {
   return f2_pack(r0, r1);
 }
 
-// Two non-negative floats -> bf16x2 with integer ops (ALU pipe, keeping the
-// special-function pipe free for exponentials): adding 0x8000 to the bit
-// pattern rounds the magnitude to the nearest bf16 (ties upward), then prmt
-// keeps the two high halves (lo in bits 0-15).
-__device__ __forceinline__ uint32_t pack_bf16x2_pos(float lo, float hi) {
-  const uint32_t a = __float_as_uint(lo) + 0x8000u;
-  const uint32_t b = __float_as_uint(hi) + 0x8000u;
+// Two floats rounded to nearest-even bf16 and packed (lo in bits 0-15) by
+// one cvt.rn.bf16x2.f32.
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
   uint32_t d;
-  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(d) : "r"(a), "r"(b));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
   return d;
 }
 
