@@ -186,6 +186,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int yq = sp / p.Wb, xq = sp % p.Wb;
   const int64_t row = static_cast<int64_t>(bh) * p.nQB + tq * HbWb + sp;
   const int32_t* blist = p.blk_idx + row * p.kmax;
+  // the first two kept block ids go out with the count instead of after it (a
+  // second L2 round trip before the first copies); only the second half of a
+  // split unit, whose list starts further on, reloads them
+  int pre0 = blist[0];
+  int pre1 = p.kmax > 1 ? blist[1] : 0;
   int n = p.blk_cnt[row];
   if (n < 0 || n > p.kmax) {
     if (threadIdx.x == 0) atomicOr(p.err, DEVERR_BOUNDS);
@@ -198,6 +203,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     } else {
       blist += h0;
       n -= h0;
+      pre0 = n > 0 ? blist[0] : 0;
+      pre1 = n > 1 ? blist[1] : 0;
     }
   }
   const int64_t begin = p.kv_begin[b], end = p.kv_end[b];
@@ -245,7 +252,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // thread 0 is also the Q/K producer: it initialises the barriers and starts
     // the Q and first K copies right away, so their latency overlaps the
     // tensor-memory allocation and the CTA-wide barrier
-    const int first_blk = n > 0 ? blist[0] : 0;
+    const int first_blk = pre0;
     for (int i = 0; i < B_COUNT; ++i)
       mbar_init(bar(i), (i >= B_P_FULL && i < B_P_FULL + S_BUFS) ? SOFTMAX_THREADS : 1u);
     *abort_flag = 0;
@@ -273,7 +280,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // ------------------------------------------------------------ Q + K producer
     if (lane == 0 && n > 0) {
       int issued_k = 1;                           // Q and K_0 went out before the CTA barrier
-      int next_blk = n > 1 ? checked(blist[1]) : 0;
+      int next_blk = n > 1 ? checked(pre1) : 0;
       for (int j = 1; j < n; ++j) {
         const int blk = next_blk;
         if (j + 1 < n) next_blk = checked(blist[j + 1]);
@@ -296,7 +303,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // ------------------------------------------------------------ V producer
     if (lane == 0 && n > 0) {
       int issued_v = 0;
-      int next_blk = checked(blist[0]);
+      int next_blk = checked(pre0);
       for (int j = 0; j < n; ++j) {
         const int blk = next_blk;
         if (j + 1 < n) next_blk = checked(blist[j + 1]);
@@ -382,8 +389,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint64_t sc2 = f2_pack(scale, scale);
     float m_run = -INFINITY, l_run = 0.f;         // running max (log2 units) and sum
     bool done = n > 0;
-    int next_blk = n > 0 ? checked(blist[0]) : 0;
-    int raw_blk = n > 1 ? blist[1] : 0;
+    int next_blk = n > 0 ? checked(pre0) : 0;
+    int raw_blk = pre1;
     // token-level window of this row's query token (a key token is visible iff
     // its y and x lie in these ranges)
     int wy0 = 0, wy1 = 0, wx0 = 0, wx1 = 0;
