@@ -51,21 +51,23 @@ ingest_kernel(const __grid_constant__ IngestParams p) {
   static_assert(NV * INGEST_THREADS == 128 * VPT, "block must split evenly");
   __shared__ double part[INGEST_WARPS][D];
 
-  int64_t unit = blockIdx.x;
+  // 32-bit index arithmetic (the grid is below 2^31 blocks): every thread
+  // derives its block before it can issue a load
+  int unit = static_cast<int>(blockIdx.x);
   int which = 0;
   while (which < 2 && unit >= p.t[which].units) {
-    unit -= p.t[which].units;
+    unit -= static_cast<int>(p.t[which].units);
     ++which;
   }
   const IngestTensor& tt = p.t[which];
   const int HbWb = p.Hb * p.Wb;
   const int nb = tt.nT - tt.tb_first;
-  const int sp = static_cast<int>(unit % HbWb);
-  int64_t rest = unit / HbWb;
-  const int tb = tt.tb_first + static_cast<int>(rest % nb);
+  const int sp = unit % HbWb;
+  int rest = unit / HbWb;
+  const int tb = tt.tb_first + rest % nb;
   rest /= nb;
-  const int h = static_cast<int>(rest % p.H);
-  const int bn = static_cast<int>(rest / p.H);
+  const int h = rest % p.H;
+  const int bn = rest / p.H;
   const int yb = sp / p.Wb, xb = sp % p.Wb;
   const int f0 = tt.T - 2 * tt.nT + 2 * tb;                     // older frame (-1: missing)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -87,13 +89,17 @@ ingest_kernel(const __grid_constant__ IngestParams p) {
 
   if (tt.copy_dst != nullptr) {
     const int64_t cb = bn + p.stream_offset;
-    const int64_t abs0 = p.first_abs[bn];
+    // ring slots of the block's two frames, once per thread (the host passes
+    // first_abs in [0, cap), so the frame numbers fit in 32 bits)
+    const int abs0 = static_cast<int>(p.first_abs[bn]);
+    const int slot_old = f0 >= 0 ? (abs0 + f0) % p.cap : 0;
+    const int slot_new = (abs0 + f0 + 1) % p.cap;
 #pragma unroll
     for (int u = 0; u < NV; ++u) {
       const int tok = (u * INGEST_THREADS + tid) / VPT;
       const int f = f0 + (tok >> 6);
       if (f < 0) continue;
-      const int64_t slot = (abs0 + f) % p.cap;
+      const int64_t slot = (tok >> 6) ? slot_new : slot_old;
       const int64_t row = ((cb * p.H + h) * p.cap + slot) * p.Y + 8 * yb + ((tok >> 3) & 7);
       *reinterpret_cast<uint4*>(tt.copy_dst + (row * p.X + 8 * xb + (tok & 7)) * D + vec * 8) = raw[u];
     }
