@@ -96,7 +96,8 @@ __device__ __forceinline__ StreamGeom stream_geom(const SelectParams& p, int b, 
   StreamGeom g;
   const int64_t begin = p.kv_begin[b], end = p.kv_end[b];
   g.m_first = begin >> 1;
-  g.slot0 = static_cast<int>(g.m_first % p.cap_blk);
+  // the host passes begin in [0, cap), so the oldest block's slot is its index
+  g.slot0 = static_cast<int>(g.m_first);
   const int nKT = static_cast<int>((end >> 1) - g.m_first);
   g.tq_kv = nKT - p.nQT + tq;
   g.ncand = (g.tq_kv + 1) * p.Hb * p.Wb;
@@ -175,7 +176,7 @@ score_kernel(const __grid_constant__ SelectParams p) {
     const int j = c0 + cc;
     if (cc < ncur) {
       const int tk = j / HbWb, spk = j - tk * HbWb;
-      const int slot = (g.slot0 + tk) % p.cap_blk;
+      const int slot = g.slot0 + tk < p.cap_blk ? g.slot0 + tk : g.slot0 + tk - p.cap_blk;
       const double2* src = reinterpret_cast<const double2*>(
           p.k_pool + ((static_cast<int64_t>(bh) * p.cap_blk + slot) * HbWb + spk) * D);
 #pragma unroll
@@ -211,18 +212,25 @@ score_kernel(const __grid_constant__ SelectParams p) {
     s3 = __dadd_rn(s3, __dmul_rn(qs[(r0 + 3) * D + c], kv));
   }
   const int j = c0 + cc;
-  const int spk = j % HbWb;
-  const int yk = spk / p.Wb, xk = spk - yk * p.Wb;
+  int yk = 0, xk = 0;
+  if (p.window > 0) {
+    const int spk = j % HbWb;
+    yk = spk / p.Wb;
+    xk = spk - yk * p.Wb;
+  }
   const double sv[4] = {s0, s1, s2, s3};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = r0 + i;
     if (r >= nrows) break;
     const int sp = sp0 + r;
-    int y0, y1, x0, x1;
-    window_bounds(sp / p.Wb, p.Hb, p.window, p.window_mode, y0, y1);
-    window_bounds(sp % p.Wb, p.Wb, p.window, p.window_mode, x0, x1);
-    const bool ok = yk >= y0 && yk < y1 && xk >= x0 && xk < x1;
+    bool ok = true;   // without a window every causal candidate is allowed
+    if (p.window > 0) {
+      int y0, y1, x0, x1;
+      window_bounds(sp / p.Wb, p.Hb, p.window, p.window_mode, y0, y1);
+      window_bounds(sp % p.Wb, p.Wb, p.window, p.window_mode, x0, x1);
+      ok = yk >= y0 && yk < y1 && xk >= x0 && xk < x1;
+    }
     // adding +0.0 turns -0.0 into +0.0, so equal scores get equal keys
     const double sc = __dadd_rn(__ddiv_rn(sv[i], p.sqrt_d), 0.0);
     const int64_t row = static_cast<int64_t>(bh) * nQB + tq * HbWb + sp;
@@ -243,20 +251,23 @@ topk_warp_kernel(const __grid_constant__ SelectParams p) {
   const int HbWb = p.Hb * p.Wb;
   const int nQB = p.nQT * HbWb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * TKW_WARPS + warp;
-  if (row >= static_cast<int64_t>(p.B) * p.H * nQB) return;
-  const int bh = static_cast<int>(row / nQB);
-  const int qi = static_cast<int>(row % nQB);
-  const int tq = qi / HbWb, sp = qi % HbWb;
+  const int64_t row64 = static_cast<int64_t>(blockIdx.x) * TKW_WARPS + warp;
+  if (row64 >= static_cast<int64_t>(p.B) * p.H * nQB) return;
+  const int row = static_cast<int>(row64);   // rows < 2^31 (checked on the host)
+  const int bh = row / nQB;
+  const int qi = row - bh * nQB;
+  const int tq = qi / HbWb, sp = qi - tq * HbWb;
   const StreamGeom g = stream_geom(p, bh / p.H, tq);
   const int ncand = g.ncand;
   if (ncand > 32 * KPL) {
     if (lane == 0) atomicOr(p.err, DEVERR_BOUNDS);
     return;
   }
-  int y0, y1, x0, x1;
-  window_bounds(sp / p.Wb, p.Hb, p.window, p.window_mode, y0, y1);
-  window_bounds(sp % p.Wb, p.Wb, p.window, p.window_mode, x0, x1);
+  int y0 = 0, y1 = p.Hb, x0 = 0, x1 = p.Wb;
+  if (p.window > 0) {
+    window_bounds(sp / p.Wb, p.Hb, p.window, p.window_mode, y0, y1);
+    window_bounds(sp % p.Wb, p.Wb, p.window, p.window_mode, x0, x1);
+  }
   const int C = (g.tq_kv + 1) * (y1 - y0) * (x1 - x0);
   int K;
   if (p.top_k > 0) {
@@ -265,7 +276,7 @@ topk_warp_kernel(const __grid_constant__ SelectParams p) {
     const double kd = ceil(__dmul_rn(p.density, static_cast<double>(C)));
     K = min(C, max(1, static_cast<int>(kd)));
   }
-  const uint64_t* krow = p.keys + row * p.c_stride;
+  const uint64_t* krow = p.keys + static_cast<int64_t>(row) * p.c_stride;
   const int nslots = (ncand + 31) / 32;
   uint32_t hi[KPL], lo[KPL];
   int lc = 0;
@@ -356,7 +367,7 @@ topk_warp_kernel(const __grid_constant__ SelectParams p) {
   for (int i = 0; i < KPL; ++i)
     if (i < nslots) lc += ((static_cast<uint64_t>(hi[i]) << 32) | lo[i]) > k_hi;
   const int need = K - __reduce_add_sync(0xffffffffu, lc);
-  int32_t* out = p.blk_idx + row * p.kmax;
+  int32_t* out = p.blk_idx + static_cast<int64_t>(row) * p.kmax;
   const uint32_t lt_mask = (1u << lane) - 1u;
   int n_band = 0, n_sel = 0;
 #pragma unroll
