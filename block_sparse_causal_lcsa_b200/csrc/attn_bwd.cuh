@@ -172,19 +172,21 @@ struct BwdLayout {
   static constexpr int SMEM_KV = KV_BAR + 256 + 1024;
 };
 
-// Ring slots of a key block's two frames (a one-frame block loads its frame twice).
+// Ring slots of a key block's two frames (a one-frame block loads its frame
+// twice). The host passes begin in [0, cap), so the frame numbers lie in
+// [0, 2 cap) and a slot is a conditional subtract; 32-bit arithmetic only.
 __device__ __forceinline__ void bwd_key_coords(const BwdParams& p, int b, int blk, int& x8, int& y8, int& s0,
                                                int& s1) {
   const int HbWb = p.Hb * p.Wb;
-  const int64_t begin = p.kv_begin[b];
-  const int tk = blk / HbWb, spk = blk % HbWb;
-  const int64_t m = (begin >> 1) + tk;
-  const int64_t a1 = 2 * m + 1;
-  const int64_t a0 = (2 * m < begin) ? a1 : 2 * m;
-  s0 = static_cast<int>(a0 % p.cap);
-  s1 = static_cast<int>(a1 % p.cap);
-  x8 = 8 * (spk % p.Wb);
-  y8 = 8 * (spk / p.Wb);
+  const int begin = static_cast<int>(p.kv_begin[b]);
+  const int tk = blk / HbWb, spk = blk - tk * HbWb;
+  const int a1 = 2 * ((begin >> 1) + tk) + 1;
+  const int a0 = a1 - 1 < begin ? a1 : a1 - 1;
+  s0 = a0 >= p.cap ? a0 - p.cap : a0;
+  s1 = a1 >= p.cap ? a1 - p.cap : a1;
+  const int yb = spk / p.Wb;
+  x8 = 8 * (spk - yb * p.Wb);
+  y8 = 8 * yb;
 }
 
 template <int D>
@@ -346,12 +348,13 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       // right after S_j and dP_j, so it runs while the elementwise warps work on
       // block j.
       auto issue_dq = [&](int jj) {
-        const uint32_t ka = sbase + L::DQ_K + (jj & 1) * L::TILE;
+        // one descriptor per operand; a step's is the base plus its byte offset / 16
+        const uint64_t kd = desc_sw128(sbase + L::DQ_K + (jj & 1) * L::TILE, L::CHUNK, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           // A = dS (16 keys = 8 packed columns), B = K: 16 keys = 16 rows of 128 bytes,
           // 64-channel columns 16 KB apart
-          bwd_umma_ts(tmem + DQ_COL, tmem + DS_COL + kk * 8, desc_sw128(ka + kk * 2048, L::CHUNK, 1024), ID_DQ,
+          bwd_umma_ts(tmem + DQ_COL, tmem + DS_COL + kk * 8, kd + kk * (2048 >> 4), ID_DQ,
                       (jj > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(bar(DQB_DQ_DONE));
@@ -364,18 +367,18 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         // S_j and dP_j overwrite what the elementwise warps read for block j-1
         if (j > 0 && !(ok = wait_bounded(bar(DQB_G_FULL), (j - 1) & 1, w))) break;
         tc_fence_after();
-        const uint32_t ka = sbase + L::DQ_K + st * L::TILE, va = sbase + L::DQ_V + st * L::TILE;
+        const uint64_t qd = desc_sw128(sbase + L::DQ_Q, 16, 1024), od = desc_sw128(sbase + L::DQ_DO, 16, 1024);
+        const uint64_t kd = desc_sw128(sbase + L::DQ_K + st * L::TILE, 16, 1024);
+        const uint64_t vd = desc_sw128(sbase + L::DQ_V + st * L::TILE, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::CHUNK + (kk & 3) * 32;
-          umma_ss(tmem, desc_sw128(sbase + L::DQ_Q + off, 16, 1024), desc_sw128(ka + off, 16, 1024), ID_SS,
-                  kk > 0 ? 1u : 0u);
+          const uint32_t off16 = ((kk >> 2) * L::CHUNK + (kk & 3) * 32) >> 4;
+          umma_ss(tmem, qd + off16, kd + off16, ID_SS, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::CHUNK + (kk & 3) * 32;
-          umma_ss(tmem + 128, desc_sw128(sbase + L::DQ_DO + off, 16, 1024), desc_sw128(va + off, 16, 1024), ID_SS,
-                  kk > 0 ? 1u : 0u);
+          const uint32_t off16 = ((kk >> 2) * L::CHUNK + (kk & 3) * 32) >> 4;
+          umma_ss(tmem + 128, od + off16, vd + off16, ID_SS, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(DQB_SD_FULL));
         umma_commit(bar(DQB_V_EMPTY + st));
@@ -551,29 +554,29 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (j > 0 && !(ok = wait_bounded(bar(KVB_ACC_DONE), (j - 1) & 1, w))) break;
         tc_fence_after();
         const uint32_t qa = sbase + L::KV_Q + st * L::TILE, ga = sbase + L::KV_DO + st * L::TILE;
+        // one descriptor per operand; a step's is the base plus its byte offset / 16
+        const uint64_t kd = desc_sw128(sbase + L::KV_K, 16, 1024), vd = desc_sw128(sbase + L::KV_V, 16, 1024);
+        const uint64_t qd = desc_sw128(qa, 16, 1024), gd = desc_sw128(ga, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::CHUNK + (kk & 3) * 32;
-          umma_ss(tmem, desc_sw128(sbase + L::KV_K + off, 16, 1024), desc_sw128(qa + off, 16, 1024), ID_SS,
-                  kk > 0 ? 1u : 0u);
+          const uint32_t off16 = ((kk >> 2) * L::CHUNK + (kk & 3) * 32) >> 4;
+          umma_ss(tmem, kd + off16, qd + off16, ID_SS, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::CHUNK + (kk & 3) * 32;
-          umma_ss(tmem + 128, desc_sw128(sbase + L::KV_V + off, 16, 1024), desc_sw128(ga + off, 16, 1024), ID_SS,
-                  kk > 0 ? 1u : 0u);
+          const uint32_t off16 = ((kk >> 2) * L::CHUNK + (kk & 3) * 32) >> 4;
+          umma_ss(tmem + 128, vd + off16, gd + off16, ID_SS, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(KVB_SD_FULL));
         if (!(ok = wait_bounded(bar(KVB_G_FULL), j & 1, w))) break;
         tc_fence_after();
+        const uint64_t gdm = desc_sw128(ga, L::CHUNK, 1024), qdm = desc_sw128(qa, L::CHUNK, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           // dV += P^T dO and dK += dS^T Q: A (16 queries = 8 packed columns) from tensor
           // memory; B = dO / Q, 16 queries = 16 rows of 128 bytes, 64-channel columns 16 KB apart
-          bwd_umma_ts(tmem + 256, tmem + kk * 8, desc_sw128(ga + kk * 2048, L::CHUNK, 1024), ID_ACC,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-          bwd_umma_ts(tmem + 384, tmem + 128 + kk * 8, desc_sw128(qa + kk * 2048, L::CHUNK, 1024), ID_ACC,
-                      (j > 0 || kk > 0) ? 1u : 0u);
+          bwd_umma_ts(tmem + 256, tmem + kk * 8, gdm + kk * (2048 >> 4), ID_ACC, (j > 0 || kk > 0) ? 1u : 0u);
+          bwd_umma_ts(tmem + 384, tmem + 128 + kk * 8, qdm + kk * (2048 >> 4), ID_ACC, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(bar(KVB_ACC_DONE));
         umma_commit(bar(KVB_Q_EMPTY + st));
