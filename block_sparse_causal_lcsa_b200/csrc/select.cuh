@@ -46,7 +46,7 @@ struct SelectParams {
 };
 
 __host__ __device__ constexpr size_t score_smem_bytes(int D) {
-  return sizeof(double) * (static_cast<size_t>(SC_ROWS) * D + static_cast<size_t>(SC_CANDS) * (D + 1));
+  return sizeof(double) * (static_cast<size_t>(SC_ROWS) * D + static_cast<size_t>(SC_CANDS) * (D + 2));
 }
 
 __device__ __forceinline__ uint64_t order_key(double s) {
@@ -109,7 +109,10 @@ __global__ void __launch_bounds__(SC_THREADS)
 score_kernel(const __grid_constant__ SelectParams p) {
   extern __shared__ __align__(16) double sc_smem[];
   double* qs = sc_smem;                         // [SC_ROWS][D]
-  double* ks = qs + SC_ROWS * D;                // [SC_CANDS][D+1]
+  // candidate rows padded to D + 2 doubles: 16-byte aligned for paired loads,
+  // and lanes (one candidate each) 4 banks apart, so a quarter warp's 16-byte
+  // loads hit distinct banks
+  double* ks = qs + SC_ROWS * D;                // [SC_CANDS][D+2]
 
   const int HbWb = p.Hb * p.Wb;
   const int nQB = p.nQT * HbWb;
@@ -192,8 +195,7 @@ score_kernel(const __grid_constant__ SelectParams p) {
 #pragma unroll
     for (int v = 0; v < PER_LANE; ++v) {
       const int e = v * 32 + lane;
-      ks[cc * (D + 1) + 2 * e] = buf[i][v].x;
-      ks[cc * (D + 1) + 2 * e + 1] = buf[i][v].y;
+      reinterpret_cast<double2*>(ks + cc * (D + 2))[e] = buf[i][v];
     }
   }
   __syncthreads();
@@ -201,15 +203,26 @@ score_kernel(const __grid_constant__ SelectParams p) {
   const int cc = tid % SC_CANDS;
   const int r0 = (tid / SC_CANDS) * 4;
   if (cc >= ncur) return;
-  const double* kr = ks + cc * (D + 1);
+  const double2* kr = reinterpret_cast<const double2*>(ks + cc * (D + 2));
+  const double2* q0 = reinterpret_cast<const double2*>(qs + (r0 + 0) * D);
+  const double2* q1 = reinterpret_cast<const double2*>(qs + (r0 + 1) * D);
+  const double2* q2 = reinterpret_cast<const double2*>(qs + (r0 + 2) * D);
+  const double2* q3 = reinterpret_cast<const double2*>(qs + (r0 + 3) * D);
   double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-#pragma unroll 8
-  for (int c = 0; c < D; ++c) {
-    const double kv = kr[c];
-    s0 = __dadd_rn(s0, __dmul_rn(qs[(r0 + 0) * D + c], kv));
-    s1 = __dadd_rn(s1, __dmul_rn(qs[(r0 + 1) * D + c], kv));
-    s2 = __dadd_rn(s2, __dmul_rn(qs[(r0 + 2) * D + c], kv));
-    s3 = __dadd_rn(s3, __dmul_rn(qs[(r0 + 3) * D + c], kv));
+  // channel pairs (c, c + 1) loaded together; the products are still added
+  // one channel at a time, in channel order
+#pragma unroll 2
+  for (int c2 = 0; c2 < D / 2; ++c2) {
+    const double2 kv = kr[c2];
+    const double2 a = q0[c2], b = q1[c2], cq = q2[c2], dq = q3[c2];
+    s0 = __dadd_rn(s0, __dmul_rn(a.x, kv.x));
+    s1 = __dadd_rn(s1, __dmul_rn(b.x, kv.x));
+    s2 = __dadd_rn(s2, __dmul_rn(cq.x, kv.x));
+    s3 = __dadd_rn(s3, __dmul_rn(dq.x, kv.x));
+    s0 = __dadd_rn(s0, __dmul_rn(a.y, kv.y));
+    s1 = __dadd_rn(s1, __dmul_rn(b.y, kv.y));
+    s2 = __dadd_rn(s2, __dmul_rn(cq.y, kv.y));
+    s3 = __dadd_rn(s3, __dmul_rn(dq.y, kv.y));
   }
   const int j = c0 + cc;
   int yk = 0, xk = 0;
