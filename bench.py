@@ -485,30 +485,33 @@ def run_ours(args, world, rank, local):
     # pinned host memory and O going back there, copies inside the timed region
     e2e = None
     if st.streaming:
-        # distinct pinned host chunks through lc.HostPipeline: each chunk's
+        # distinct pinned host chunks through the library's own pipeline
+        # (lcsa_pipeline_*: the C ABI takes the host buffers): each chunk's
         # inputs cross PCIe while the previous chunk computes, and its O comes
-        # back on a third stream; the timed region runs from the first timed
-        # chunk's host-to-device copy to the last chunk's device-to-host copy.
-        # No L2 flush in this loop: every step's inputs arrive by a fresh copy
-        # and its working set (cache + chunk) is larger than L2.
+        # back on a third stream; the timed region runs, on the pipeline's own
+        # events, from the first timed chunk's host-to-device copy to the last
+        # chunk's device-to-host copy. No L2 flush in this loop: every step's
+        # inputs arrive by a fresh copy and its working set (cache + chunk) is
+        # larger than L2.
         host = [tuple(t.cpu().pin_memory() for t in c) for c in st.chunks]
         ho = torch.empty(host[0][0].shape, dtype=torch.bfloat16).pin_memory()
-        pipe = lc.HostPipeline(st.step)
-        e_start = torch.cuda.Event(enable_timing=True)
-        done = None
+        pipe = lc.NativePipeline(st.step.cache, w.q_frames, st.step.params)
         for i in range(args.warmup + args.steps):
             if i == args.warmup:
-                torch.cuda.synchronize()
-                e_start.record(pipe.h2d_stream)
+                pipe.sync()
+                pipe.start_timer()
             st.step.cache.set_state(st.base_state)
-            done = pipe.submit(*host[i % len(host)], ho)
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(e_start.elapsed_time(done) / args.steps, world)
+            pipe.submit(*host[i % len(host)], ho)
+        pipe.sync()
+        e2e_ms = max_over_ranks(pipe.elapsed_ms() / args.steps, world)
+        pipe.close()
+        st.step.cache.set_state(st.base_state)
         hq, hk, hv = host[0]
         e2e = {"value": whole_job_ms_per_chunk(e2e_ms, chunks_per_step, world), "unit": UNIT,
                "h2d_bytes_per_step": hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2,
                "d2h_bytes_per_step": ho.numel() * 2,
-               "pipelined": "copies of chunk i+1 overlap the compute of chunk i (lc.HostPipeline); "
+               "api": "lcsa_pipeline_submit (C ABI, host buffers)",
+               "pipelined": "copies of chunk i+1 overlap the compute of chunk i; "
                             "%d distinct host chunks cycled; no L2 flush (inputs arrive by copy)" % len(host)}
     else:
         hq, hk, hv = st.q.cpu().pin_memory(), st.k.cpu().pin_memory(), st.v.cpu().pin_memory()

@@ -9,6 +9,7 @@ from .api import (  # noqa: F401
     HostPipeline,
     KVCache,
     LcsaError,
+    NativePipeline,
     SelectParams,
     StreamingStep,
     WINDOW_PRESERVE,

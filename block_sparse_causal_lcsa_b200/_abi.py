@@ -100,6 +100,13 @@ PROTOTYPES = {
     "lcsa_debug_set_wait_limit_ns": (C.c_int, [C.c_uint64]),
     "lcsa_debug_stalled_wait": (C.c_int, [C.c_uint64, C.c_void_p]),
     "lcsa_debug_exp2_poly": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p]),
+    "lcsa_pipeline_create": (C.c_int, [C.POINTER(KVCacheStruct), C.c_int32, C.POINTER(SelectParamsStruct),
+                                       C.POINTER(C.c_void_p)]),
+    "lcsa_pipeline_submit": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "lcsa_pipeline_sync": (C.c_int, [C.c_void_p]),
+    "lcsa_pipeline_start_timer": (C.c_int, [C.c_void_p]),
+    "lcsa_pipeline_elapsed_ms": (C.c_int, [C.c_void_p, C.POINTER(C.c_float)]),
+    "lcsa_pipeline_destroy": (None, [C.c_void_p]),
 }
 
 

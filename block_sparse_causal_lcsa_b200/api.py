@@ -455,6 +455,51 @@ class StreamingStep:
         return self.o, self.lse
 
 
+class NativePipeline:
+    """The library's streaming pipeline (lcsa_pipeline_*): chunks of Q, K, V
+    from pinned host tensors, the step (ingest, select, attention) and O back
+    to a pinned host tensor, with the copies of one chunk overlapping the
+    steps of its neighbours, all queued by the C library on its own streams.
+    It owns its device buffers and advances `cache` (whose state it shares)
+    chunk by chunk. Host tensors must stay untouched until `sync()`."""
+
+    def __init__(self, cache: "KVCache", q_frames: int, params: SelectParams):
+        self.cache = cache          # the pipeline holds a pointer to cache.struct
+        self.shape = (cache.B, cache.H, q_frames, cache.Y, cache.X, cache.D)
+        h = C.c_void_p()
+        _check(_lib.lcsa_pipeline_create(C.byref(cache.struct), q_frames, C.byref(params.struct()), C.byref(h)),
+               "lcsa_pipeline_create")
+        self._h = h
+
+    def submit(self, hq: torch.Tensor, hk: torch.Tensor, hv: torch.Tensor, ho: torch.Tensor) -> None:
+        for t in (hq, hk, hv, ho):
+            if t.is_cuda or not t.is_pinned() or not t.is_contiguous() or t.dtype != torch.bfloat16:
+                raise ValueError("NativePipeline takes contiguous pinned bf16 host tensors")
+            if tuple(t.shape) != self.shape:
+                raise ValueError("expected host tensors of shape %s" % (self.shape,))
+        _check(_lib.lcsa_pipeline_submit(self._h, hq.data_ptr(), hk.data_ptr(), hv.data_ptr(), ho.data_ptr()),
+               "lcsa_pipeline_submit")
+
+    def sync(self) -> None:
+        _check(_lib.lcsa_pipeline_sync(self._h), "lcsa_pipeline_sync")
+
+    def start_timer(self) -> None:
+        _check(_lib.lcsa_pipeline_start_timer(self._h), "lcsa_pipeline_start_timer")
+
+    def elapsed_ms(self) -> float:
+        ms = C.c_float()
+        _check(_lib.lcsa_pipeline_elapsed_ms(self._h, C.byref(ms)), "lcsa_pipeline_elapsed_ms")
+        return float(ms.value)
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            _lib.lcsa_pipeline_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+
 class HostPipeline:
     """Streams chunks from pinned host memory through a StreamingStep, with the
     copies of one chunk overlapping the compute of its neighbours (a streaming

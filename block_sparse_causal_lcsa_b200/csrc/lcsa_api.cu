@@ -879,3 +879,5 @@ lcsa_status lcsa_debug_set_wait_limit_ns(uint64_t ns) {
 }
 
 }  // extern "C"
+
+#include "pipeline.cuh"

@@ -454,6 +454,49 @@ LCSA_API lcsa_status lcsa_debug_stalled_wait(uint64_t limit_ns, lcsa_stream_t st
 LCSA_API lcsa_status lcsa_debug_exp2_poly(const float* x, float* y, int64_t n,
                                           lcsa_stream_t stream);
 
+/*
+ * Streaming pipeline (section 3: the model runs as a stream, 8 video frames =
+ * 2 latent frames per chunk, with a KV cache): chunks come from host memory
+ * and their outputs go back there, with the copies of one chunk overlapping
+ * the step of its neighbours.
+ *
+ * lcsa_pipeline_create - a pipeline over the caller's cache `kv`, chunks of
+ *   q_frames frames per stream, selection parameters `params` (kmax is
+ *   computed here, params->kmax is ignored; a token-level window mode also
+ *   sets the attention's token window). The pipeline allocates, on the
+ *   current device, two device input sets (Q, K, V), the step's scratch and O;
+ *   lcsa_pipeline_destroy frees them. kv must stay valid, and must not be
+ *   used by other calls, while the pipeline exists: each submit advances its
+ *   host-side state as lcsa_ingest_chunk does. Errors: as check of kv,
+ *   LCSA_ERR_SHAPE for q_frames outside [1, cap_frames], LCSA_ERR_INVALID_ARG
+ *   for a bad window mode, LCSA_ERR_CUDA if an allocation fails (nothing is
+ *   then kept). *out receives the pipeline, or NULL on error.
+ * lcsa_pipeline_submit - queue one chunk: q_host, k_host, v_host each hold
+ *   [B][H][q_frames][Y][X][D] bf16, contiguous, in host memory; o_host receives
+ *   O in the same layout. Per chunk: three host-to-device copies on an upload
+ *   stream, then lcsa_ingest_chunk, lcsa_select_blocks and
+ *   lcsa_sparse_attn_fwd_ex on a compute stream, then the device-to-host copy
+ *   of O on a read-back stream, all ordered by events; it returns once the
+ *   work is queued. For the copies to overlap the steps the host buffers must
+ *   be page-locked (cudaHostAlloc or cudaHostRegister). Host inputs must stay
+ *   unchanged, and o_host unread, until lcsa_pipeline_sync returns. Call from
+ *   the device the pipeline was created on (else LCSA_ERR_INVALID_ARG).
+ * lcsa_pipeline_sync - wait for every queued chunk; returns the device error
+ *   status as lcsa_last_device_error does.
+ * lcsa_pipeline_start_timer / lcsa_pipeline_elapsed_ms - time, with events
+ *   on the pipeline's own streams, from the first upload of the next submit
+ *   to the read-back of the last chunk submitted (elapsed_ms waits for it).
+ */
+typedef struct lcsa_pipeline lcsa_pipeline;
+LCSA_API lcsa_status lcsa_pipeline_create(lcsa_kv_cache* kv, int32_t q_frames,
+                                          const lcsa_select_params* params, lcsa_pipeline** out);
+LCSA_API lcsa_status lcsa_pipeline_submit(lcsa_pipeline* pl, const void* q_host, const void* k_host,
+                                          const void* v_host, void* o_host);
+LCSA_API lcsa_status lcsa_pipeline_sync(lcsa_pipeline* pl);
+LCSA_API lcsa_status lcsa_pipeline_start_timer(lcsa_pipeline* pl);
+LCSA_API lcsa_status lcsa_pipeline_elapsed_ms(lcsa_pipeline* pl, float* ms);
+LCSA_API void lcsa_pipeline_destroy(lcsa_pipeline* pl);
+
 #ifdef __cplusplus
 }
 #endif

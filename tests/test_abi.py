@@ -115,6 +115,33 @@ def test_attention_rejects_caches_of_2_22_key_blocks(lib):
     assert lib.lcsa_sparse_attn_fwd(*args) == _abi.ERR_SHAPE
 
 
+def test_pipeline_argument_errors(lib):
+    """lcsa_pipeline_* reject bad arguments before any device allocation or
+    copy (only invalid requests here: a valid one would allocate)."""
+    from block_sparse_causal_lcsa_b200 import _abi
+    kv = _abi.KVCacheStruct()
+    kv.k, kv.v, kv.k_pool = 0x1000, 0x2000, 0x3000
+    kv.B, kv.H, kv.cap_frames, kv.Y, kv.X, kv.D = 1, 1, 6, 16, 16, 128
+    sp = _abi.SelectParamsStruct(0, 0, 0, 0, 0.136, 1e-5)
+    h = C.c_void_p(0x1)
+    assert lib.lcsa_pipeline_create(C.byref(kv), 2, C.byref(sp), None) == _abi.ERR_INVALID_ARG
+    assert lib.lcsa_pipeline_create(C.byref(kv), 2, None, C.byref(h)) == _abi.ERR_INVALID_ARG
+    assert h.value is None                                            # *out cleared on error
+    assert lib.lcsa_pipeline_create(C.byref(kv), 0, C.byref(sp), C.byref(h)) == _abi.ERR_SHAPE
+    assert lib.lcsa_pipeline_create(C.byref(kv), 8, C.byref(sp), C.byref(h)) == _abi.ERR_SHAPE   # > cap
+    sp.window_mode = 7
+    assert lib.lcsa_pipeline_create(C.byref(kv), 2, C.byref(sp), C.byref(h)) == _abi.ERR_INVALID_ARG
+    sp.window_mode = 0
+    kv.cap_frames = 5                                                 # odd capacity
+    assert lib.lcsa_pipeline_create(C.byref(kv), 2, C.byref(sp), C.byref(h)) == _abi.ERR_SHAPE
+    assert lib.lcsa_pipeline_submit(None, 0x1000, 0x1000, 0x1000, 0x1000) == _abi.ERR_INVALID_ARG
+    assert lib.lcsa_pipeline_sync(None) == _abi.ERR_INVALID_ARG
+    assert lib.lcsa_pipeline_start_timer(None) == _abi.ERR_INVALID_ARG
+    ms = C.c_float()
+    assert lib.lcsa_pipeline_elapsed_ms(None, C.byref(ms)) == _abi.ERR_INVALID_ARG
+    lib.lcsa_pipeline_destroy(None)                                   # no-op
+
+
 def test_select_kmax_host_rule(lib):
     from block_sparse_causal_lcsa_b200 import _abi
     kv = _abi.KVCacheStruct()

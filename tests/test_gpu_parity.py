@@ -280,6 +280,41 @@ def test_host_pipeline_equals_eager_steps(lc):
     assert torch.equal(caches[0].k_pool, caches[1].k_pool)
 
 
+def test_native_pipeline_equals_eager_steps(lc):
+    """Six chunks from pinned host memory through the library's pipeline
+    (lcsa_pipeline_*: uploads, step and read-back on its own streams) against
+    the same chunks stepped eagerly from device memory: identical outputs,
+    cache contents and cache state; the pipeline's timer covers the run."""
+    w = li.Workload("nativepipe", B=2, H=2, D=128, Y=16, X=24, q_frames=2, kv_past=(0, 0), cap_frames=6,
+                    density=0.4, seed=95)
+    caches = [lc.KVCache(w.B, w.H, w.cap_frames, w.Y, w.X, w.D) for _ in range(2)]
+    for c in caches:
+        c.k.zero_(), c.v.zero_(), c.k_pool.zero_()
+    step = lc.StreamingStep(caches[0], 2, params_of(lc, w))
+    pipe = lc.NativePipeline(caches[1], 2, params_of(lc, w))
+    g = torch.Generator().manual_seed(9)
+    shp = (w.B, w.H, 2, w.Y, w.X, w.D)
+    chunks = [tuple(torch.randn(shp, generator=g).to(torch.bfloat16).pin_memory() for _ in range(3))
+              for _ in range(6)]
+    outs = [torch.empty(shp, dtype=torch.bfloat16).pin_memory() for _ in range(6)]
+    pipe.start_timer()
+    for t, c in enumerate(chunks):
+        pipe.submit(*c, outs[t])
+    pipe.sync()
+    assert pipe.elapsed_ms() > 0.0
+    for t, c in enumerate(chunks):
+        o, _ = step(*(x.cuda() for x in c))
+        torch.cuda.synchronize()
+        assert torch.equal(o.cpu(), outs[t]), "chunk %d" % t
+    assert lc.last_device_error() == 0
+    assert caches[0].state() == caches[1].state()
+    assert torch.equal(caches[0].k, caches[1].k) and torch.equal(caches[0].v, caches[1].v)
+    assert torch.equal(caches[0].k_pool, caches[1].k_pool)
+    with pytest.raises(ValueError):
+        pipe.submit(chunks[0][0].cuda(), *chunks[0][1:], outs[0])
+    pipe.close()
+
+
 def test_host_pipeline_rejects_device_and_pageable_tensors(lc):
     cache = lc.KVCache(1, 1, 4, 8, 8, 128)
     step = lc.StreamingStep(cache, 2, lc.SelectParams(top_k=1))
