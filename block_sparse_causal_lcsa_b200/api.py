@@ -60,14 +60,76 @@ def pooled_shape(x: torch.Tensor) -> Tuple[int, ...]:
     return (B, H, (T + 1) // 2, Y // 8, X // 8, D)
 
 
+def _check_tokens(name: str, t) -> None:
+    """A token tensor [B][H][T][Y][X][D] in bf16 (its device is checked with
+    the call's other tensors)."""
+    if not isinstance(t, torch.Tensor) or t.dim() != 6 or t.dtype != torch.bfloat16:
+        raise ValueError("%s must be a bf16 tensor [B][H][T][Y][X][D]" % name)
+
+
+def _check_buffer(name: str, t, dtype: torch.dtype, shape) -> None:
+    """A buffer the library takes as a bare pointer and sizes from its other
+    arguments: any other dtype, shape or layout would let a kernel read or
+    write past it (ValueError, nothing launched)."""
+    if not isinstance(t, torch.Tensor):
+        raise ValueError("%s must be a tensor" % name)
+    if t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def _check_workspace(t) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor")
+
+
+def _check_device(dev: torch.device, **tensors) -> None:
+    """All tensors of a call in the memory of the one GPU it runs on (the
+    kernels dereference their pointers there). None entries are skipped."""
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("%s must be a CUDA tensor, got %s" % (name, t.device))
+        if t.device != dev:
+            raise ValueError("%s must be on %s with the call's other tensors, got %s" % (name, dev, t.device))
+
+
+def _query_blocks(q: torch.Tensor) -> int:
+    _, _, T, Y, X, _ = q.shape
+    return ((T + 1) // 2) * (Y // 8) * (X // 8)
+
+
+def _check_block_lists(q: torch.Tensor, blk_idx, blk_cnt) -> None:
+    """blk_idx int32 [B,H,nQB,kmax] and blk_cnt int32 [B,H,nQB] for the query
+    chunk q (nQB = ceil(T/2) * Y/8 * X/8); kmax is blk_idx's last extent."""
+    if not isinstance(blk_idx, torch.Tensor) or blk_idx.dim() != 4:
+        raise ValueError("blk_idx must be an int32 tensor [B,H,nQB,kmax]")
+    B, H = q.shape[0], q.shape[1]
+    nQB = _query_blocks(q)
+    _check_buffer("blk_idx", blk_idx, torch.int32, (B, H, nQB, blk_idx.shape[-1]))
+    _check_buffer("blk_cnt", blk_cnt, torch.int32, (B, H, nQB))
+
+
 def pool_qk(q: torch.Tensor, k: Optional[torch.Tensor] = None,
             q_pool: Optional[torch.Tensor] = None, k_pool: Optional[torch.Tensor] = None,
             stream: Optional[torch.cuda.Stream] = None):
     """Mean-pool Q (and K) over 2x8x8 token blocks into float64 features."""
+    _check_tokens("q", q)
+    if k is not None:
+        _check_tokens("k", k)
     if q_pool is None:
         q_pool = torch.empty(pooled_shape(q), dtype=torch.float64, device=q.device)
+    else:
+        _check_buffer("q_pool", q_pool, torch.float64, pooled_shape(q))
     if k is not None and k_pool is None:
         k_pool = torch.empty(pooled_shape(k), dtype=torch.float64, device=k.device)
+    elif k is not None:
+        _check_buffer("k_pool", k_pool, torch.float64, pooled_shape(k))
+    _check_device(q.device, q=q, k=k, q_pool=q_pool, k_pool=k_pool if k is not None else None)
     qd = tensor_desc(q)
     kd = tensor_desc(k) if k is not None else None
     _check(_lib.lcsa_pool_qk(C.byref(qd), C.byref(kd) if kd is not None else None,
@@ -89,9 +151,12 @@ class KVCache:
         self.k_pool = (k_pool if k_pool is not None else
                        torch.empty((B, H, cap_frames // 2, Y // 8, X // 8, D), dtype=torch.float64,
                                    device=device))
-        for t in (self.k, self.v, self.k_pool):
-            if not t.is_contiguous():
-                raise ValueError("cache buffers must be contiguous")
+        pool_shape = (B, H, cap_frames // 2, Y // 8, X // 8, D)
+        for name, t, dtype, shp in (("k", self.k, torch.bfloat16, shape), ("v", self.v, torch.bfloat16, shape),
+                                    ("k_pool", self.k_pool, torch.float64, pool_shape)):
+            _check_buffer(name, t, dtype, shp)
+            if t.device != self.k.device:
+                raise ValueError("k, v and k_pool must be on one device")
         self.struct = _abi.KVCacheStruct()
         self.struct.k = self.k.data_ptr()
         self.struct.v = self.v.data_ptr()
@@ -138,9 +203,12 @@ def kv_append(cache: KVCache, k_new: torch.Tensor, v_new: torch.Tensor,
               stream: Optional[torch.cuda.Stream] = None) -> None:
     """Append a chunk to streams [offset, offset+B) of the cache. Without
     k_pool_new the call pools K itself while copying it (one read of K)."""
+    _check_tokens("k_new", k_new)
+    _check_tokens("v_new", v_new)
+    if k_pool_new is not None:
+        _check_buffer("k_pool_new", k_pool_new, torch.float64, pooled_shape(k_new))
+    _check_device(cache.k.device, cache=cache.k, k_new=k_new, v_new=v_new, k_pool_new=k_pool_new)
     kd, vd = tensor_desc(k_new), tensor_desc(v_new)
-    if k_pool_new is not None and (not k_pool_new.is_contiguous() or k_pool_new.dtype != torch.float64):
-        raise ValueError("k_pool_new must be contiguous float64")
     _check(_lib.lcsa_kv_append(C.byref(cache.struct), C.byref(kd), C.byref(vd),
                                k_pool_new.data_ptr() if k_pool_new is not None else None,
                                stream_offset, _stream(stream)),
@@ -152,8 +220,14 @@ def ingest_chunk(q: torch.Tensor, cache: KVCache, k_new: torch.Tensor, v_new: to
                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """pool_qk(q) and kv_append(cache, k_new, v_new) (K pooled on the way) in
     one launch; returns q_pool."""
+    _check_tokens("q", q)
     if q_pool is None:
         q_pool = torch.empty(pooled_shape(q), dtype=torch.float64, device=q.device)
+    else:
+        _check_buffer("q_pool", q_pool, torch.float64, pooled_shape(q))
+    _check_tokens("k_new", k_new)
+    _check_tokens("v_new", v_new)
+    _check_device(cache.k.device, cache=cache.k, q=q, k_new=k_new, v_new=v_new, q_pool=q_pool)
     qd, kd, vd = tensor_desc(q), tensor_desc(k_new), tensor_desc(v_new)
     _check(_lib.lcsa_ingest_chunk(C.byref(qd), q_pool.data_ptr(), C.byref(cache.struct), C.byref(kd), C.byref(vd),
                                   stream_offset, _stream(stream)), "lcsa_ingest_chunk")
@@ -194,18 +268,8 @@ def _check_select_io(q_pool: torch.Tensor, q_frames: int, cache: KVCache, kmax: 
             "blk_idx": (blk_idx, torch.int32, (cache.B, cache.H, nQB, kmax)),
             "blk_cnt": (blk_cnt, torch.int32, (cache.B, cache.H, nQB))}
     for name, (t, dtype, shape) in want.items():
-        if not isinstance(t, torch.Tensor):
-            raise ValueError("%s must be a tensor" % name)
-        if t.dtype != dtype:
-            raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
-        if tuple(t.shape) != shape:
-            raise ValueError("%s must have shape %s for this cache, got %s" % (name, shape, tuple(t.shape)))
-        if not t.is_contiguous():
-            raise ValueError("%s must be contiguous" % name)
-    dev = cache.k.device
-    for name, (t, _, _) in want.items():
-        if not t.is_cuda or t.device != dev:
-            raise ValueError("%s must be a CUDA tensor on the cache's device %s, got %s" % (name, dev, t.device))
+        _check_buffer(name, t, dtype, shape)
+    _check_device(cache.k.device, cache=cache.k, q_pool=q_pool, blk_idx=blk_idx, blk_cnt=blk_cnt)
 
 
 def select_blocks(q_pool: torch.Tensor, q_frames: int, cache: KVCache, params: SelectParams,
@@ -225,8 +289,9 @@ def select_blocks(q_pool: torch.Tensor, q_frames: int, cache: KVCache, params: S
     need = select_workspace_bytes(cache, q_frames)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-    elif not workspace.is_cuda or workspace.device != cache.k.device or not workspace.is_contiguous():
-        raise ValueError("workspace must be a contiguous CUDA tensor on the cache's device")
+    else:
+        _check_workspace(workspace)
+        _check_device(cache.k.device, workspace=workspace)
     sp = params.struct(kmax)
     _check(_lib.lcsa_select_blocks(q_pool.data_ptr(), q_frames, C.byref(cache.struct), C.byref(sp),
                                    blk_idx.data_ptr(), blk_cnt.data_ptr(), workspace.data_ptr(),
@@ -267,12 +332,18 @@ def sparse_attn_fwd(q: torch.Tensor, cache: KVCache, blk_idx: torch.Tensor, blk_
     the key tokens inside its window. With a ``workspace`` (see
     attn_workspace), a partly empty last wave of CTAs is evened out by splitting
     its query blocks in two (lcsa_sparse_attn_fwd_ex)."""
+    _check_tokens("q", q)
     if o is None:
         o = torch.empty_like(q)
+    _check_tokens("o", o)
     if lse is None and with_lse:
         lse = torch.empty(q.shape[:5], dtype=torch.float32, device=q.device)
-    if not blk_idx.is_contiguous() or not blk_cnt.is_contiguous():
-        raise ValueError("blk_idx and blk_cnt must be contiguous")
+    _check_block_lists(q, blk_idx, blk_cnt)
+    if lse is not None:
+        _check_buffer("lse", lse, torch.float32, q.shape[:5])
+    if workspace is not None:
+        _check_workspace(workspace)
+    _check_device(q.device, q=q, cache=cache.k, o=o, lse=lse, blk_idx=blk_idx, blk_cnt=blk_cnt, workspace=workspace)
     qd, od = tensor_desc(q), tensor_desc(o)
     lse_ptr = lse.data_ptr() if lse is not None else None
     if workspace is not None:
@@ -305,6 +376,12 @@ def segment_blocks(q_frames: int, cache: KVCache, kmax: Optional[int] = None,
                    stream: Optional[torch.cuda.Stream] = None):
     """Block lists for dense attention inside each stream (segment) of the cache:
     (blk_idx [B,H,nQB,kmax], blk_cnt [B,H,nQB]) for sparse_attn_fwd / _bwd."""
+    if blk_idx is not None:
+        if not isinstance(blk_idx, torch.Tensor) or blk_idx.dim() != 4:
+            raise ValueError("blk_idx must be an int32 tensor [B,H,nQB,kmax]")
+        if kmax is not None and kmax != blk_idx.shape[-1]:
+            raise ValueError("kmax %d differs from blk_idx's last extent %d" % (kmax, blk_idx.shape[-1]))
+        kmax = blk_idx.shape[-1]
     if kmax is None:
         kmax = int(_lib.lcsa_segment_kmax(C.byref(cache.struct)))
     nQB = ((q_frames + 1) // 2) * (cache.Y // 8) * (cache.X // 8)
@@ -313,6 +390,9 @@ def segment_blocks(q_frames: int, cache: KVCache, kmax: Optional[int] = None,
         blk_idx = torch.empty((cache.B, cache.H, nQB, kmax), dtype=torch.int32, device=dev)
     if blk_cnt is None:
         blk_cnt = torch.empty((cache.B, cache.H, nQB), dtype=torch.int32, device=dev)
+    _check_buffer("blk_idx", blk_idx, torch.int32, (cache.B, cache.H, nQB, kmax))
+    _check_buffer("blk_cnt", blk_cnt, torch.int32, (cache.B, cache.H, nQB))
+    _check_device(dev, cache=cache.k, blk_idx=blk_idx, blk_cnt=blk_cnt)
     _check(_lib.lcsa_segment_blocks(q_frames, C.byref(cache.struct), blk_idx.shape[-1], blk_idx.data_ptr(),
                                     blk_cnt.data_ptr(), _stream(stream)), "lcsa_segment_blocks")
     return blk_idx, blk_cnt
@@ -330,18 +410,25 @@ def sparse_attn_bwd(q: torch.Tensor, cache: KVCache, blk_idx: torch.Tensor, blk_
     """Gradients of sparse_attn_fwd for the same selection: (dq like q, dk and
     dv in the cache layout [B][H][cap][Y][X][D]). dk / dv default to zeros, so
     ring slots outside the cached frames read as zero."""
+    for name, t in (("q", q), ("o", o), ("d_o", d_o)):
+        _check_tokens(name, t)
     if dq is None:
         dq = torch.empty_like(q)
+    _check_tokens("dq", dq)
     if dk is None:
         dk = torch.zeros_like(cache.k)
     if dv is None:
         dv = torch.zeros_like(cache.v)
-    need = sparse_attn_bwd_workspace_bytes(cache, q.shape[2])
+    _check_block_lists(q, blk_idx, blk_cnt)
+    _check_buffer("lse", lse, torch.float32, q.shape[:5])
+    _check_buffer("dk", dk, torch.bfloat16, cache.k.shape)
+    _check_buffer("dv", dv, torch.bfloat16, cache.v.shape)
     if workspace is None:
+        need = sparse_attn_bwd_workspace_bytes(cache, q.shape[2])
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    for t in (blk_idx, blk_cnt, lse, dk, dv):
-        if not t.is_contiguous():
-            raise ValueError("blk_idx, blk_cnt, lse, dk and dv must be contiguous")
+    _check_workspace(workspace)
+    _check_device(q.device, q=q, cache=cache.k, o=o, d_o=d_o, dq=dq, lse=lse, dk=dk, dv=dv, blk_idx=blk_idx,
+                  blk_cnt=blk_cnt, workspace=workspace)
     qd, od, gd, dqd = tensor_desc(q), tensor_desc(o), tensor_desc(d_o), tensor_desc(dq)
     _check(_lib.lcsa_sparse_attn_bwd(C.byref(qd), C.byref(cache.struct), blk_idx.data_ptr(), blk_cnt.data_ptr(),
                                      blk_idx.shape[-1], C.byref(od), lse.data_ptr(), C.byref(gd), C.byref(dqd),

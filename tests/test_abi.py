@@ -262,3 +262,82 @@ def test_binding_rejects_bad_selection_outputs(lib):
             with pytest.raises(ValueError):
                 lc.select_blocks(a["q_pool"], 2, cache, params, a["blk_idx"].shape[-1], a["blk_idx"],
                                  a["blk_cnt"], workspace=torch.zeros(16, dtype=torch.uint8))
+
+
+def test_binding_rejects_bad_buffers_of_every_call(lib):
+    """Every binding call that hands the library a bare pointer checks the
+    buffer's dtype, shape and layout against what the call derives from its
+    other arguments, then that all tensors sit on one GPU, before calling the
+    library (ValueError naming the argument, nothing launched). On this host
+    the all-good case stops at the device check."""
+    import torch
+    import block_sparse_causal_lcsa_b200 as lc
+
+    bf, f32, f64, i32 = torch.bfloat16, torch.float32, torch.float64, torch.int32
+    cache = lc.KVCache(1, 2, 6, 16, 24, 128, device="cpu")
+    cache.struct.begin[0], cache.struct.end[0] = 0, 6
+    q = torch.zeros((1, 2, 2, 16, 24, 128), dtype=bf)
+    nQB, kmax = 1 * 2 * 3, 5
+    idx, cnt = torch.zeros((1, 2, nQB, kmax), dtype=i32), torch.zeros((1, 2, nQB), dtype=i32)
+    lse = torch.zeros((1, 2, 2, 16, 24), dtype=f32)
+    ws = torch.zeros(64, dtype=torch.uint8)
+    qp = torch.zeros((1, 2, 1, 2, 3, 128), dtype=f64)
+
+    def fwd(**kw):
+        a = dict(q=q, blk_idx=idx, blk_cnt=cnt, o=torch.empty_like(q), lse=lse, workspace=ws)
+        a.update(kw)
+        lc.sparse_attn_fwd(a["q"], cache, a["blk_idx"], a["blk_cnt"], a["o"], a["lse"], workspace=a["workspace"])
+
+    cases = [
+        (lambda: fwd(blk_idx=idx.long()), r"blk_idx must be torch\.int32"),
+        (lambda: fwd(blk_idx=idx[0]), r"blk_idx must be an int32 tensor"),
+        (lambda: fwd(blk_idx=idx[:, :, 1:]), r"blk_idx must have shape"),
+        (lambda: fwd(blk_idx=torch.zeros((1, 2, kmax, nQB), dtype=i32).transpose(2, 3)), r"blk_idx must be contiguous"),
+        (lambda: fwd(blk_cnt=cnt.long()), r"blk_cnt must be torch\.int32"),
+        (lambda: fwd(blk_cnt=cnt[:, :, 1:]), r"blk_cnt must have shape"),
+        (lambda: fwd(lse=lse.double()), r"lse must be torch\.float32"),
+        (lambda: fwd(lse=lse[:, :, :1]), r"lse must have shape"),
+        (lambda: fwd(o=torch.empty_like(q, dtype=f32)), r"o must be a bf16 tensor"),
+        (lambda: fwd(q=q.float()), r"q must be a bf16 tensor"),
+        (lambda: fwd(workspace=ws[::2]), r"workspace must be a contiguous"),
+        (lambda: fwd(), r"q must be a CUDA tensor"),
+        # backward: gradient buffers in the cache layout, the forward's LSE
+        (lambda: lc.sparse_attn_bwd(q, cache, idx, cnt, q, lse, q, torch.empty_like(q),
+                                    torch.zeros((1, 2, 4, 16, 24, 128), dtype=bf), torch.zeros_like(cache.v), ws),
+         r"dk must have shape"),
+        (lambda: lc.sparse_attn_bwd(q, cache, idx, cnt, q, lse, q, torch.empty_like(q), torch.zeros_like(cache.k),
+                                    torch.zeros_like(cache.v, dtype=f32), ws), r"dv must be torch\.bfloat16"),
+        (lambda: lc.sparse_attn_bwd(q, cache, idx, cnt, q, lse.half(), q, torch.empty_like(q),
+                                    torch.zeros_like(cache.k), torch.zeros_like(cache.v), ws), r"lse must be torch\.float32"),
+        (lambda: lc.sparse_attn_bwd(q, cache, idx, cnt, q, lse, q.float(), torch.empty_like(q),
+                                    torch.zeros_like(cache.k), torch.zeros_like(cache.v), ws), r"d_o must be a bf16"),
+        (lambda: lc.sparse_attn_bwd(q, cache, idx.long(), cnt, q, lse, q, torch.empty_like(q),
+                                    torch.zeros_like(cache.k), torch.zeros_like(cache.v), ws), r"blk_idx must be torch\.int32"),
+        (lambda: lc.sparse_attn_bwd(q, cache, idx, cnt, q, lse, q, torch.empty_like(q), torch.zeros_like(cache.k),
+                                    torch.zeros_like(cache.v), ws), r"q must be a CUDA tensor"),
+        # pooling, ingest and append: pooled rows [B,H,ceil(T/2),Y/8,X/8,D] in float64
+        (lambda: lc.pool_qk(q, None, qp.float()), r"q_pool must be torch\.float64"),
+        (lambda: lc.pool_qk(q, None, qp[:, :1]), r"q_pool must have shape"),
+        (lambda: lc.pool_qk(q, q, qp, torch.zeros((1, 2, 2, 2, 3, 128), dtype=f64)), r"k_pool must have shape"),
+        (lambda: lc.pool_qk(q, None, qp), r"q must be a CUDA tensor"),
+        (lambda: lc.ingest_chunk(q, cache, q, q, torch.zeros((1, 2, 1, 2, 3, 64), dtype=f64)), r"q_pool must have shape"),
+        (lambda: lc.ingest_chunk(q, cache, q, q.float(), qp), r"v_new must be a bf16"),
+        (lambda: lc.ingest_chunk(q, cache, q, q, qp), r"cache must be a CUDA tensor"),
+        (lambda: lc.kv_append(cache, q, q, qp.float()), r"k_pool_new must be torch\.float64"),
+        (lambda: lc.kv_append(cache, q, q, torch.zeros((1, 2, 2, 2, 3, 128), dtype=f64)), r"k_pool_new must have shape"),
+        (lambda: lc.kv_append(cache, q, q), r"cache must be a CUDA tensor"),
+        # segment lists: kmax is blk_idx's last extent
+        (lambda: lc.segment_blocks(2, cache, kmax + 1, idx, cnt), r"kmax 6 differs"),
+        (lambda: lc.segment_blocks(2, cache, None, idx, cnt.long()), r"blk_cnt must be torch\.int32"),
+        (lambda: lc.segment_blocks(2, cache, None, idx, cnt), r"cache must be a CUDA tensor"),
+        # caller-given cache buffers
+        (lambda: lc.KVCache(1, 2, 6, 16, 24, 128, device="cpu", k=torch.zeros((1, 2, 4, 16, 24, 128), dtype=bf)),
+         r"k must have shape"),
+        (lambda: lc.KVCache(1, 2, 6, 16, 24, 128, device="cpu",
+                            k_pool=torch.zeros((1, 2, 3, 2, 3, 128), dtype=f32)), r"k_pool must be torch\.float64"),
+        (lambda: lc.KVCache(1, 2, 6, 16, 24, 128, device="cpu",
+                            v=torch.zeros((1, 2, 6, 16, 128, 24), dtype=bf).transpose(4, 5)), r"v must be contiguous"),
+    ]
+    for call, msg in cases:
+        with pytest.raises(ValueError, match=msg):
+            call()

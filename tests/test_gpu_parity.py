@@ -463,6 +463,19 @@ def test_out_of_range_block_id_is_reported(lc):
     assert lc.last_device_error() == -8
 
 
+def test_host_buffer_is_rejected_before_launch(lc):
+    """A host-memory LSE buffer beside a chunk on the GPU: the binding raises
+    ValueError before the library is called, and no device error follows."""
+    w = li.workload("tiny")
+    x = li.make_inputs(w)
+    g = run_gpu(lc, w, x)
+    step = g["step"]
+    host_lse = torch.zeros(tuple(g["q"].shape[:5]), dtype=torch.float32)
+    with pytest.raises(ValueError, match="lse must be a CUDA tensor"):
+        lc.sparse_attn_fwd(g["q"], g["cache"], step.blk_idx, step.blk_cnt, lse=host_lse)
+    assert lc.last_device_error() == 0
+
+
 def test_exp2_polynomial_error_bound(lc):
     """The FMA-pipe 2^x that the softmax can use in place of the
     special-function unit stays within its fitted relative error bound (7.5e-5, plus float32 rounding)
