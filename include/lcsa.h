@@ -481,11 +481,20 @@ LCSA_API lcsa_status lcsa_debug_exp2_poly(const float* x, float* y, int64_t n,
  *   be page-locked (cudaHostAlloc or cudaHostRegister). Host inputs must stay
  *   unchanged, and o_host unread, until lcsa_pipeline_sync returns. Call from
  *   the device the pipeline was created on (else LCSA_ERR_INVALID_ARG).
+ *   Errors: LCSA_ERR_INVALID_ARG for a NULL argument or another device (nothing
+ *   queued); LCSA_ERR_CUDA if a copy, event or stream call fails; otherwise
+ *   the first error of the step's three calls (e.g. LCSA_ERR_SHAPE for an odd
+ *   q_frames once a stream holds frames, as lcsa_ingest_chunk). After any
+ *   error other than the first kind, part of the chunk may be queued and kv
+ *   may have advanced: call lcsa_pipeline_sync, then restore kv's state or
+ *   destroy the pipeline.
  * lcsa_pipeline_sync - wait for every queued chunk; returns the device error
  *   status as lcsa_last_device_error does.
  * lcsa_pipeline_start_timer / lcsa_pipeline_elapsed_ms - time, with events
  *   on the pipeline's own streams, from the first upload of the next submit
  *   to the read-back of the last chunk submitted (elapsed_ms waits for it).
+ *   elapsed_ms returns LCSA_ERR_INVALID_ARG while start_timer has not yet
+ *   been followed by a submit, and LCSA_ERR_CUDA if no timer was started.
  */
 typedef struct lcsa_pipeline lcsa_pipeline;
 LCSA_API lcsa_status lcsa_pipeline_create(lcsa_kv_cache* kv, int32_t q_frames,
