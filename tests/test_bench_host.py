@@ -94,3 +94,28 @@ def test_allowed_pairs_equals_the_oracles_candidate_counts():
                                        window=window, mode=mode)
             want += int(Cs.sum())
         assert got == want, (window, mode, got, want)
+
+
+def test_reference_arm_prints_the_contract_line():
+    """bench.py --impl reference times the oracle on host cores and prints the
+    same JSON line as the GPU arm: the same metric, unit and workload text,
+    time-like (lower is better), an e2e that moves no bytes between host and
+    device, and a cpu_baseline describing this run. Under several ranks, rank 0
+    alone runs it; the others return without work."""
+    import argparse
+    import json
+
+    b = _bench()
+    args = argparse.Namespace(workload="chunk", steps=1, warmup=0)
+    assert b.run_reference(args, 2, 1) is None
+    line = b.run_reference(args, 1, 0)
+    json.dumps(line)
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["metric"] == b.METRIC and line["unit"] == b.UNIT
+    assert line["config"]["workload"] == b.WORKLOAD_TEXT["chunk"]
+    assert line["higher_is_better"] is False and line["value"] > 0 and line["steps"] == 1
+    assert line["e2e"] == {"value": line["value"], "unit": b.UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] > 0 and cb["sample"]
