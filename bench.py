@@ -634,6 +634,44 @@ def extra_workloads(lc, dev, peaks, args, flush_l2):
 
 
 # ----------------------------------------------------------------------------- oracle arm
+def backward_cpu_baseline(w, x, d_o, budget_s):
+    """The oracle's attention backward as it stands, timed on host cores on a
+    bounded sample: the oracle selects the blocks of head 0 of stream 0 itself,
+    then attend_rows_backward runs on its query blocks in order until the
+    budget is spent. Scaled by kept block pairs to the whole workload: K_i
+    depends only on the geometry (causality, window, density), so every head
+    of a stream keeps as many pairs as its head 0."""
+    from oracle import lcsa_oracle as orc
+
+    qh, kh, vh = orc.widen(x["q"][0, 0]), orc.widen(x["k"][0][0]), orc.widen(x["v"][0][0])
+    Tq, Y, X, D = qh.shape
+    sel, total_kept = None, 0
+    for b in range(w.B):
+        qb = qh if b == 0 else orc.widen(x["q"][b, 0])
+        kb = kh if b == 0 else orc.widen(x["k"][b][0])
+        sb, Ks, _ = orc.select_head(orc.pool_blocks(qb), orc.pool_blocks(kb), Tq, kb.shape[0], Y, X,
+                                    w.top_k, w.density, w.window, w.window_mode)
+        total_kept += int(Ks.sum()) * w.H
+        if b == 0:
+            sel = sb
+    q2, k2, v2 = qh.reshape(-1, D), kh.reshape(-1, D), vh.reshape(-1, D)
+    g2 = orc.widen(d_o[0, 0]).reshape(-1, D)
+    n_rows = kept = 0
+    with CpuMeter() as meter:
+        for i in range(len(sel)):
+            qidx = orc.block_token_index(Tq, Y, X, [i])
+            kidx = orc.block_token_index(kh.shape[0], Y, X, sel[i])
+            orc.attend_rows_backward(q2[qidx], k2[kidx], v2[kidx], g2[qidx])
+            n_rows += 1
+            kept += len(sel[i])
+            if time.perf_counter() - meter.w0 > budget_s:
+                break
+    return {"value": round(meter.wall / kept * total_kept * 1e3, 1), "unit": "ms/clip", "cores": meter.cores,
+            "cpu_model": cpu_model(), "kind": "oracle", "kept_pairs_total": total_kept,
+            "sample": "%d query blocks (%d kept block pairs) of head 0, blocks selected by the oracle, "
+                      "attend_rows_backward in fp64, scaled by kept pairs to all %d" % (n_rows, kept, total_kept)}
+
+
 def run_backward(args, world, rank, local):
     """Attention gradients for training with the block-sparse causal mask: the
     whole clip is the key timeline, the forward runs once (untimed), then each
@@ -654,7 +692,8 @@ def run_backward(args, world, rank, local):
     idx, cnt = lc.select_blocks(lc.pool_qk(q)[0], w.q_frames, cache, params)
     o, lse = lc.sparse_attn_fwd(q, cache, idx, cnt)
     g = torch.Generator().manual_seed(w.seed + 11)
-    d_o = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(dev)
+    d_o_host = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    d_o = d_o_host.to(dev)
     dq, dk, dv = torch.empty_like(q), torch.zeros_like(cache.k), torch.zeros_like(cache.v)
     ws = torch.empty(max(lc.sparse_attn_bwd_workspace_bytes(cache, w.q_frames), 16), dtype=torch.uint8, device=dev)
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
@@ -706,33 +745,7 @@ def run_backward(args, world, rank, local):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        from oracle import lcsa_oracle as orc
-        t0 = time.perf_counter()
-        c0 = time.process_time()
-        h = 0
-        qh, kh, vh = orc.widen(x["q"][0, h]), orc.widen(x["k"][0][h]), orc.widen(x["v"][0][h])
-        sel = [idx[0, h, i, :int(cnt[0, h, i])].cpu().numpy() for i in range(cnt.shape[2])]
-        # a bounded sample: the first query blocks of one head, scaled by their share of the kept pairs
-        n_rows = 0
-        kept = 0
-        Tq, Y, X, D = qh.shape
-        for i in range(len(sel)):
-            qidx = orc.block_token_index(Tq, Y, X, [i])
-            kidx = orc.block_token_index(kh.shape[0], Y, X, sel[i])
-            orc.attend_rows_backward(qh.reshape(-1, D)[qidx], kh.reshape(-1, D)[kidx], vh.reshape(-1, D)[kidx],
-                                     orc.widen(d_o[0, h].cpu()).reshape(-1, D)[qidx])
-            n_rows += 1
-            kept += len(sel[i])
-            if time.perf_counter() - t0 > args.cpu_budget:
-                break
-        el = time.perf_counter() - t0
-        cpu_used = time.process_time() - c0
-        total_kept = int(cnt.sum().item())
-        cpu_ms = el / kept * total_kept * 1e3
-        line["cpu_baseline"] = {"value": round(cpu_ms, 1), "unit": "ms/clip", "cores": round(cpu_used / el, 2),
-                                "cpu_model": cpu_model(), "kind": "oracle",
-                                "sample": "%d query blocks (%d kept block pairs) of head 0, attend_rows_backward "
-                                          "in fp64, scaled by kept pairs to all %d" % (n_rows, kept, total_kept)}
+        line["cpu_baseline"] = backward_cpu_baseline(w, x, d_o_host, args.cpu_budget)
     return line
 
 

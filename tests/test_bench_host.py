@@ -119,3 +119,24 @@ def test_reference_arm_prints_the_contract_line():
     assert line["e2e"] == {"value": line["value"], "unit": b.UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] > 0 and cb["sample"]
+
+
+def test_backward_cpu_baseline_selects_with_the_oracle():
+    """The backward mode's CPU baseline runs on host inputs alone: the oracle
+    selects its own blocks, and the kept-pair total it scales by equals every
+    head's own count times the heads (K_i depends only on the geometry)."""
+    import lcsa_inputs as li
+    from oracle import lcsa_oracle as orc
+
+    b = _bench()
+    w = li.small_variant(li.workload("clip"), H=2, Y=16, X=24)
+    x = li.make_inputs(w)
+    d_o = torch.randn(x["q"].shape, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    cb = b.backward_cpu_baseline(w, x, d_o, budget_s=1.0)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["unit"] == "ms/clip" and cb["cores"] > 0
+    assert w.B == 1
+    for h in range(w.H):
+        qh, kh = orc.widen(x["q"][0, h]), orc.widen(x["k"][0][h])
+        _, Ks, _ = orc.select_head(orc.pool_blocks(qh), orc.pool_blocks(kh), qh.shape[0], kh.shape[0], w.Y, w.X,
+                                   w.top_k, w.density, w.window, w.window_mode)
+        assert int(Ks.sum()) * w.H == cb["kept_pairs_total"]
