@@ -1,5 +1,7 @@
 """GPU parity of the attention gradients (lcsa_sparse_attn_bwd) against the
-fp64 oracle's attend_head_backward, on the selections the library made.
+fp64 oracle's attend_head_backward. The oracle works from the host inputs
+alone: it pools and selects its own blocks, and each case first checks that
+the library attended exactly those blocks over the same cached key frames.
 
 Tolerance (derived from the arithmetic): Q, K, V, dO are bf16 and exact in
 both paths; the GPU rounds P and dS to bf16 (relative error 2^-9) before their
@@ -14,6 +16,7 @@ import pytest
 import torch
 
 import lcsa_inputs as li
+from lcsa_harness import check_selection, oracle_head
 from oracle import lcsa_oracle as orc
 
 pytestmark = pytest.mark.gpu
@@ -57,11 +60,20 @@ def _run(lc, w, x, seed=1):
     idx, cnt = lc.select_blocks(q_pool, w.q_frames, cache, params)
     o, lse = lc.sparse_attn_fwd(q, cache, idx, cnt)
     g = torch.Generator().manual_seed(seed)
-    d_o = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(dev)
-    dq, dk, dv = lc.sparse_attn_bwd(q, cache, idx, cnt, o, lse, d_o)
+    d_o_host = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    dq, dk, dv = lc.sparse_attn_bwd(q, cache, idx, cnt, o, lse, d_o_host.to(dev))
     torch.cuda.synchronize()
     assert lc.last_device_error() == 0
-    return cache, q, idx, cnt, d_o, dq, dk, dv
+    return cache, q, idx, cnt, d_o_host, dq, dk, dv
+
+
+def _oracle_grads(w, x, d_o, b, h):
+    """Stream b, head h through the oracle from the host inputs alone: its own
+    selection, the key timeline, and dq, dk, dv over that timeline."""
+    ref = oracle_head(w, x, b, h, rows=[])    # pooling and selection; no forward rows
+    kh, vh = orc.widen(x["k"][b][h]), orc.widen(x["v"][b][h])
+    rq, rk, rv = orc.attend_head_backward(orc.widen(x["q"][b, h]), kh, vh, ref["sel"], orc.widen(d_o[b, h]))
+    return ref["sel"], kh, rq, rk, rv
 
 
 def _logical(cache, t, b, h):
@@ -75,12 +87,11 @@ def _compare(lc, w, x, heads=None):
     worst = [0.0, 0.0, 0.0]
     for b in range(w.B):
         for h in (range(w.H) if heads is None else heads):
-            lo, hi = cache.state()[b]
-            kh = _logical(cache, cache.k, b, h)
-            vh = _logical(cache, cache.v, b, h)
-            sel = [idx[b, h, i, :int(cnt[b, h, i])].cpu().numpy() for i in range(cnt.shape[2])]
-            rq, rk, rv = orc.attend_head_backward(orc.widen(q[b, h].cpu()), kh, vh, sel, orc.widen(d_o[b, h].cpu()))
             where = "%s b%d h%d" % (w.name, b, h)
+            sel, kh, rq, rk, rv = _oracle_grads(w, x, d_o, b, h)
+            # the library attended the oracle's blocks over the same key frames
+            check_selection(idx[b, h].cpu().numpy(), cnt[b, h].cpu().numpy(), sel, where)
+            assert np.array_equal(_logical(cache, cache.k, b, h), kh), where + " cached K"
             e = [_check(dq[b, h].double().cpu().numpy(), rq, where + " dq")[0],
                  _check(_logical(cache, dk, b, h), rk, where + " dk")[0],
                  _check(_logical(cache, dv, b, h), rv, where + " dv")[0]]

@@ -367,22 +367,28 @@ def test_fused_append_equals_pool_then_append(lc, cap, chunks):
     b = lc.KVCache(2, H, cap, Y, X, D)
     for c in (a, b):
         c.k.zero_(), c.v.zero_(), c.k_pool.zero_()
+    timeline = [[None] * H for _ in range(2)]   # the oracle's cache of each (stream, head)
     for t in chunks:
-        k = (torch.randn((2, H, t, Y, X, D), generator=g) * 3).to(torch.bfloat16).cuda()
+        k_host = (torch.randn((2, H, t, Y, X, D), generator=g) * 3).to(torch.bfloat16)
+        k = k_host.cuda()
         v = torch.randn((2, H, t, Y, X, D), generator=g).to(torch.bfloat16).cuda()
         lc.kv_append(a, k, v)
         lc.kv_append(b, k, v, lc.pool_qk(k)[0])
         assert a.state() == b.state()
+        for s_ in range(2):
+            for h in range(H):
+                timeline[s_][h] = orc.kv_append(timeline[s_][h], orc.widen(k_host[s_, h]), cap)
     torch.cuda.synchronize()
     assert lc.last_device_error() == 0
     assert torch.equal(a.k, b.k) and torch.equal(a.v, b.v)
     assert torch.equal(a.k_pool, b.k_pool)
-    # and the pooled rows are the oracle's means of the cached frames
+    # and the ring holds the oracle's cache, with the oracle's means of it as pooled rows
     for s_ in range(2):
         for h in range(H):
             lo, hi = a.state()[s_]
             frames = torch.stack([a.k[s_, h, f % cap].cpu() for f in range(lo, hi)])
-            ref = orc.pool_blocks(orc.widen(frames))
+            assert np.array_equal(frames.double().numpy(), timeline[s_][h])
+            ref = orc.pool_blocks(timeline[s_][h])
             assert np.array_equal(ring_to_logical(a, a.k_pool.cpu().numpy(), s_, h), ref)
 
 

@@ -48,12 +48,11 @@ def test_segment_lists_forward_and_backward(lc, w):
     x, cache, q, idx, cnt = _setup(lc, w)
     o, lse = lc.sparse_attn_fwd(q, cache, idx, cnt)
     g = torch.Generator().manual_seed(5)
-    d_o = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    d_o = torch.randn(q.shape, generator=g).to(torch.bfloat16)   # host; the oracle reads this copy
     Tq = w.q_frames
     for b, F in enumerate(w.seg_frames):
         d_o[b, :, :Tq - F] = 0          # padding rows carry no gradient
-    d_o = d_o.cuda()
-    dq, dk, dv = lc.sparse_attn_bwd(q, cache, idx, cnt, o, lse, d_o)
+    dq, dk, dv = lc.sparse_attn_bwd(q, cache, idx, cnt, o, lse, d_o.cuda())
     torch.cuda.synchronize()
     assert lc.last_device_error() == 0
     Hb, Wb = w.Y // 8, w.X // 8
@@ -72,7 +71,7 @@ def test_segment_lists_forward_and_backward(lc, w):
             ro, rl = orc.segment_attention(qs, ks, vs)
             check_output(o[b, h, Tq - F:].double().cpu().numpy(), ro, lse[b, h, Tq - F:].double().cpu().numpy(), rl,
                          "%s b%d h%d" % (w.name, b, h))
-            rq, rk, rv = orc.segment_attention_backward(qs, ks, vs, orc.widen(d_o[b, h, Tq - F:].cpu()))
+            rq, rk, rv = orc.segment_attention_backward(qs, ks, vs, orc.widen(d_o[b, h, Tq - F:]))
             for got, ref, name in ((dq[b, h, Tq - F:].double().cpu().numpy(), rq, "dq"),
                                    (_ring(cache, dk, b, h), rk, "dk"), (_ring(cache, dv, b, h), rv, "dv")):
                 rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
