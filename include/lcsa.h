@@ -381,6 +381,8 @@ LCSA_API lcsa_status lcsa_sparse_attn_fwd_ex(const lcsa_tensor* q, const lcsa_kv
  * the backward). blk_idx [B][H][nQB][kmax], blk_cnt [B][H][nQB] as for
  * lcsa_select_blocks; kmax >= lcsa_segment_kmax(kv), else LCSA_ERR_CAPACITY.
  * The lists feed lcsa_sparse_attn_fwd / lcsa_sparse_attn_bwd unchanged.
+ * lcsa_segment_kmax returns the number of key blocks of the longest segment
+ * (its temporal blocks x Y/8 x X/8), or 0 for a NULL or invalid kv.
  */
 LCSA_API int32_t lcsa_segment_kmax(const lcsa_kv_cache* kv);
 LCSA_API lcsa_status lcsa_segment_blocks(int32_t q_frames, const lcsa_kv_cache* kv, int32_t kmax,
