@@ -3,7 +3,8 @@
 Each function takes torch CUDA tensors, marshals their pointers, extents and
 strides into the C structs of include/lcsa.h and calls the entry point of the
 same name on the current torch stream. Output buffers are allocated with torch
-when the caller does not pass them (the library itself allocates nothing).
+when the caller does not pass them (the library itself allocates nothing,
+except the buffers a NativePipeline owns).
 No step of the attention path runs here: there is no CPU fallback, and a
 missing or incomplete liblcsa.so raises ImportError at import.
 """

@@ -20,9 +20,12 @@
  * Conventions
  * - Memory: the caller owns every buffer. The library allocates no device or
  *   host memory (the attention kernel allocates tensor memory on the SM for
- *   its own lifetime only). Its only device state is a per-device error word
- *   and the fixed scratch array of lcsa_select_blocks_noalloc. A call writes
- *   only its output arguments (and that array).
+ *   its own lifetime only), except the streaming pipeline: lcsa_pipeline_create
+ *   allocates its input sets, scratch, O and streams, and
+ *   lcsa_pipeline_destroy frees them. Its only other device state is a
+ *   per-device error word and the fixed scratch array of
+ *   lcsa_select_blocks_noalloc. A call writes only its output arguments (and
+ *   that array).
  * - Pointers named "device" must be CUDA device pointers on the current
  *   device; all others are host pointers.
  * - Errors: argument and shape errors are returned synchronously, before any
