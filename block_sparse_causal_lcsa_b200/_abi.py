@@ -117,7 +117,10 @@ def load(path: str = LIB_PATH) -> C.CDLL:
             "or __graft_entry__.build()" % path)
     lib = C.CDLL(path)
     for name, (res, args) in PROTOTYPES.items():
-        fn = getattr(lib, name)  # AttributeError if the library lacks an entry point
+        try:
+            fn = getattr(lib, name)
+        except AttributeError:
+            raise ImportError("%s lacks the entry point %s (stale or foreign build)" % (path, name)) from None
         fn.restype = res
         fn.argtypes = args
     if lib.lcsa_abi_version() != 1:

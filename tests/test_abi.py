@@ -341,3 +341,14 @@ def test_binding_rejects_bad_buffers_of_every_call(lib):
     for call, msg in cases:
         with pytest.raises(ValueError, match=msg):
             call()
+
+
+def test_missing_or_incomplete_library_fails_loudly():
+    """No silent fallback: a missing liblcsa.so, or a shared library without
+    its entry points, raises ImportError at load."""
+    import _ctypes
+    from block_sparse_causal_lcsa_b200 import _abi
+    with pytest.raises(ImportError, match="not built"):
+        _abi.load("/nonexistent/liblcsa.so")
+    with pytest.raises(ImportError, match="lacks the entry point lcsa_"):
+        _abi.load(_ctypes.__file__)     # a real shared library with none of them
